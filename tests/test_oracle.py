@@ -1,0 +1,289 @@
+"""Pins of the CPU oracle against facts fixed by the pages and by mathematics
+(no GPU). Source: "Transformers are SSMs: Generalized Models and Efficient
+Algorithms Through Structured State Space Duality"."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.signal
+
+import oracle
+import ssd_inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def tiny(T=48, H=4, P=3, N=5, G=2, b=2, seed=0, init=False, D=True, varlen=None, **kw):
+    """Small random problem (float32 values, not bf16-rounded)."""
+    rng = np.random.default_rng(seed)
+    tot = T * b
+    if varlen is not None:
+        b, tot = 1, int(sum(varlen))
+    f = np.float32
+    inp = {
+        "x": rng.standard_normal((b, tot // b, H, P)).astype(f),
+        "dt": (rng.standard_normal((b, tot // b, H)) - 1.0).astype(f),
+        "A_log": rng.uniform(-1.0, 1.0, H).astype(f),
+        "B": rng.standard_normal((b, tot // b, G, N)).astype(f),
+        "C": rng.standard_normal((b, tot // b, G, N)).astype(f),
+        "D": rng.standard_normal(H).astype(f) if D else None,
+        "initial_states": None,
+        "cu_seqlens": None,
+        "dt_softplus": True,
+    }
+    nseq = b
+    if varlen is not None:
+        inp["cu_seqlens"] = np.concatenate([[0], np.cumsum(varlen)]).astype(np.int32)
+        nseq = len(varlen)
+    if init:
+        inp["initial_states"] = rng.standard_normal((nseq, H, P, N)).astype(f)
+    inp.update(kw)
+    return inp
+
+
+def rel_err(a, b):
+    return float(np.max(np.abs(a - b)) / max(np.max(np.abs(b)), 1e-300))
+
+
+# ---------------------------------------------------------------- golden values
+
+def _golden_inp(case):
+    T = len(case["dt"])
+    P, N = case["P"], case["N"]
+    A_log = {"log(ln(2)/2)": math.log(math.log(2) / 2), "0": 0.0,
+             "log(ln(2))": math.log(math.log(2))}[case["A_log_expr"]]
+    inp = {
+        "x": np.array(case["x"], dtype=np.float32).reshape(1, T, 1, P),
+        "dt": np.array(case["dt"], dtype=np.float32).reshape(1, T, 1),
+        "A_log": np.array([A_log], dtype=np.float32),
+        "B": np.array(case["B"], dtype=np.float32).reshape(1, T, 1, N),
+        "C": np.array(case["C"], dtype=np.float32).reshape(1, T, 1, N),
+        "D": np.array([case["D"]], dtype=np.float32),
+        "initial_states": None if case["h0"] is None else np.full((1, 1, P, N), case["h0"], np.float32),
+        "cu_seqlens": None,
+        "dt_softplus": case["dt_softplus"],
+    }
+    return inp
+
+
+@pytest.mark.parametrize("idx", [0, 1, 2])
+def test_golden_hand_worked(idx):
+    """Hand-worked values of the recurrence (tests/golden/scalar_recurrence.json)."""
+    case = json.load(open(os.path.join(GOLDEN, "scalar_recurrence.json")))["cases"][idx]
+    inp = _golden_inp(case)
+    y, fin = oracle.recurrence(inp)
+    ln2 = math.log(2.0)
+    if "y_ln2" in case:
+        want_y = np.array([c0 + c1 * ln2 for c0, c1 in case["y_ln2"]])
+        want_f = case["final_ln2"][0] + case["final_ln2"][1] * ln2
+    else:
+        want_y = np.array(case["y"], dtype=np.float64)
+        want_f = np.array(case["final"], dtype=np.float64)
+    # A_log is stored in float32, so a = 1/2 holds to ~1e-7 relative
+    np.testing.assert_allclose(y.reshape(want_y.shape), want_y, rtol=2e-6, atol=1e-6)
+    np.testing.assert_allclose(fin.reshape(np.shape(want_f)), want_f, rtol=2e-6, atol=1e-6)
+
+
+# ---------------------------------------------------- brute-force quadratic form
+
+@pytest.mark.parametrize("init,D", [(False, True), (True, True), (True, False)])
+def test_recurrence_equals_quadratic_form(init, D):
+    """Sec. 3.4.2 / 5.1: the SSM equals multiplication by the explicit semiseparable M."""
+    inp = tiny(T=40, H=4, P=3, N=5, G=2, b=2, init=init, D=D, seed=1)
+    y_rec, _ = oracle.recurrence(inp)
+    y_quad = oracle.quadratic_form(inp)
+    assert rel_err(y_rec, y_quad) < 1e-12
+
+
+def test_recurrence_equals_quadratic_form_varlen():
+    inp = tiny(H=2, P=2, N=3, G=1, varlen=[7, 1, 20, 12], init=True, seed=2)
+    y_rec, _ = oracle.recurrence(inp)
+    assert rel_err(y_rec, oracle.quadratic_form(inp)) < 1e-12
+
+
+def test_impulse_columns_match_semiseparable_matrix():
+    """Column j of M is the response to a unit input at time j (one channel)."""
+    T, N = 24, 4
+    inp = tiny(T=T, H=1, P=1, N=N, G=1, b=1, D=False, seed=3)
+    M = oracle.semiseparable_matrix(inp, 0, 0)
+    cols = []
+    for j in range(T):
+        e = np.zeros_like(inp["x"])
+        e[0, j, 0, 0] = 1.0
+        y, _ = oracle.recurrence(dict(inp, x=e))
+        cols.append(y[0, :, 0, 0])
+    M_imp = np.stack(cols, axis=1)
+    assert rel_err(M_imp, M) < 1e-12
+    # Def. 3.1: every block on or below the diagonal has rank <= N
+    for i0 in (8, 12, 17):
+        blk = M_imp[i0:, :i0]
+        s = np.linalg.svd(blk, compute_uv=False)
+        assert np.sum(s > 1e-9 * s[0]) <= N
+
+
+# ------------------------------------------------------------------ closed forms
+
+def test_decay_one_is_causal_linear_attention():
+    """a == 1 (A_log = -inf, so A = -0): masked attention with the all-ones causal
+    mask, i.e. a cumulative sum over time (Sec. 4.2 / 5.2)."""
+    inp = tiny(T=33, H=2, P=3, N=4, G=1, b=1, init=True, seed=4)
+    inp["A_log"] = np.full(2, -np.inf, dtype=np.float32)
+    y, fin = oracle.recurrence(inp)
+    delta, a = oracle.discretize(inp)
+    assert np.all(a == 1.0)
+    x = inp["x"][0].astype(np.float64)
+    Bm = inp["B"][0, :, 0].astype(np.float64)
+    Cm = inp["C"][0, :, 0].astype(np.float64)
+    for h in range(2):
+        kv = np.einsum("tp,tn->tpn", delta[:, h, None] * x[:, h], Bm)
+        S = np.cumsum(kv, axis=0) + inp["initial_states"][0, h][None].astype(np.float64)
+        want = np.einsum("tpn,tn->tp", S, Cm) + float(inp["D"][h]) * x[:, h]
+        assert rel_err(y[0, :, h], want) < 1e-12
+        assert rel_err(fin[0, h], S[-1]) < 1e-12
+
+
+def test_decay_zero_keeps_only_the_diagonal():
+    """a == 0 (A_log = +30 underflows exp(delta * A) to 0): y_t = (C_t . B_t) delta_t x_t + D x_t."""
+    inp = tiny(T=20, H=2, P=3, N=4, G=2, b=1, init=True, seed=5)
+    inp["A_log"] = np.full(2, 30.0, dtype=np.float32)
+    y, _ = oracle.recurrence(inp)
+    delta, a = oracle.discretize(inp)
+    assert np.all(a == 0.0)
+    x = inp["x"][0].astype(np.float64)
+    for h in range(2):
+        g = h // 1
+        cb = np.sum(inp["C"][0, :, g].astype(np.float64) * inp["B"][0, :, g], axis=1)
+        want = (cb * delta[:, h])[:, None] * x[:, h] + float(inp["D"][h]) * x[:, h]
+        assert rel_err(y[0, :, h], want) < 1e-12
+
+
+def test_scalar_lti_is_first_order_filter():
+    """N = P = 1, B = C = 1, constant delta: y_t = a y_{t-1} + delta x_t, the textbook
+    first-order IIR filter (scipy.signal.lfilter)."""
+    T = 64
+    inp = tiny(T=T, H=1, P=1, N=1, G=1, b=1, D=False, seed=6)
+    inp["B"][:] = 1.0
+    inp["C"][:] = 1.0
+    inp["dt"][:] = 0.3
+    y, _ = oracle.recurrence(inp)
+    delta, a = oracle.discretize(inp)
+    want = scipy.signal.lfilter([delta[0, 0]], [1.0, -a[0, 0]], inp["x"][0, :, 0, 0].astype(np.float64))
+    assert rel_err(y[0, :, 0, 0], want) < 1e-12
+
+
+def test_lti_is_causal_convolution():
+    """Constant a, B, C (Sec. 2.1 LTI case): y = K * x with K_k = (C . B) a^k delta."""
+    T, N = 50, 3
+    inp = tiny(T=T, H=1, P=2, N=N, G=1, b=1, D=False, seed=7)
+    inp["dt"][:] = -0.5
+    inp["B"][:] = inp["B"][0, 0]
+    inp["C"][:] = inp["C"][0, 0]
+    y, _ = oracle.recurrence(inp)
+    delta, a = oracle.discretize(inp)
+    cb = float(inp["C"][0, 0, 0].astype(np.float64) @ inp["B"][0, 0, 0].astype(np.float64))
+    K = cb * delta[0, 0] * a[0, 0] ** np.arange(T)
+    for p in range(2):
+        want = np.convolve(K, inp["x"][0, :, 0, p].astype(np.float64))[:T]
+        assert rel_err(y[0, :, 0, p], want) < 1e-12
+
+
+# ------------------------------------------------------------------- invariants
+
+def test_split_sequence_state_passing():
+    """Sec. 8.2 (context parallelism): running [0, T/2) then [T/2, T) from the
+    first half's final state equals the whole run."""
+    inp = tiny(T=60, H=2, P=3, N=4, G=1, b=1, init=True, seed=8)
+    y, fin = oracle.recurrence(inp)
+    half = lambda a, s: None if a is None else a[:, s]
+    first = dict(inp, x=inp["x"][:, :30], dt=inp["dt"][:, :30], B=inp["B"][:, :30], C=inp["C"][:, :30])
+    y1, f1 = oracle.recurrence(first)
+    second = dict(inp, x=inp["x"][:, 30:], dt=inp["dt"][:, 30:], B=inp["B"][:, 30:], C=inp["C"][:, 30:],
+                  initial_states=f1.astype(np.float32))
+    y2, f2 = oracle.recurrence(second)
+    # f1 is rounded to float32 when passed back in: compare at float32 resolution
+    assert rel_err(np.concatenate([y1, y2], axis=1), y) < 1e-6
+    assert rel_err(f2, fin) < 1e-6
+
+
+def test_linearity_in_input_and_initial_state():
+    inp1 = tiny(T=30, H=2, P=2, N=3, G=1, b=1, init=True, D=True, seed=9)
+    inp2 = tiny(T=30, H=2, P=2, N=3, G=1, b=1, init=True, D=True, seed=10)
+    inp2.update({k: inp1[k] for k in ("dt", "A_log", "B", "C", "D")})
+    al, be = 0.75, -1.25
+    mix = dict(inp1, x=(al * inp1["x"].astype(np.float64) + be * inp2["x"]),
+               initial_states=(al * inp1["initial_states"].astype(np.float64) + be * inp2["initial_states"]))
+    # float32 inputs: keep the mixed values exactly representable by rounding first
+    mix["x"] = mix["x"].astype(np.float32)
+    mix["initial_states"] = mix["initial_states"].astype(np.float32)
+    y1, f1 = oracle.recurrence(inp1)
+    y2, f2 = oracle.recurrence(inp2)
+    ym, fm = oracle.recurrence(mix)
+    assert rel_err(ym, al * y1 + be * y2) < 1e-6
+    assert rel_err(fm, al * f1 + be * f2) < 1e-6
+
+
+def test_varlen_equals_separate_runs():
+    """Sec. 8.3: packed sequences exchange no state."""
+    lens = [5, 17, 1, 30]
+    inp = tiny(H=3, P=2, N=3, G=1, varlen=lens, init=True, seed=11)
+    y, fin = oracle.recurrence(inp)
+    cu = inp["cu_seqlens"]
+    for s in range(len(lens)):
+        a, b = cu[s], cu[s + 1]
+        one = dict(inp, x=inp["x"][:, a:b], dt=inp["dt"][:, a:b], B=inp["B"][:, a:b], C=inp["C"][:, a:b],
+                   initial_states=inp["initial_states"][s:s + 1], cu_seqlens=None)
+        ys, fs = oracle.recurrence(one)
+        assert rel_err(y[:, a:b], ys) < 1e-14
+        assert rel_err(fin[s], fs[0]) < 1e-14
+
+
+def test_empty_sequence_passes_initial_state_through():
+    inp = tiny(H=2, P=2, N=2, G=1, varlen=[4, 0, 3], init=True, seed=12)
+    _, fin = oracle.recurrence(inp)
+    np.testing.assert_array_equal(fin[1], inp["initial_states"][1].astype(np.float64))
+
+
+def test_group_mapping_is_contiguous():
+    """GVA (Sec. 7.2): head h reads B/C group h // (H / G)."""
+    inp = tiny(T=16, H=4, P=2, N=3, G=2, b=1, seed=13)
+    y, _ = oracle.recurrence(inp)
+    for h in range(4):
+        g = h // 2
+        one = dict(inp, x=inp["x"][:, :, h:h + 1], dt=inp["dt"][:, :, h:h + 1], A_log=inp["A_log"][h:h + 1],
+                   D=inp["D"][h:h + 1], B=inp["B"][:, :, g:g + 1], C=inp["C"][:, :, g:g + 1])
+        yh, _ = oracle.recurrence(one)
+        assert rel_err(y[:, :, h:h + 1], yh) < 1e-14
+
+
+def test_pairs_subset_matches_full_run():
+    inp = tiny(T=20, H=3, P=2, N=3, G=1, b=2, init=True, seed=14)
+    y, fin = oracle.recurrence(inp)
+    ys, fs = oracle.recurrence_pairs(inp, [(1, 2), (0, 1)])
+    assert np.array_equal(ys[0], y[1, :, 2])
+    assert np.array_equal(fs[1], fin[0, 1])
+
+
+# ------------------------------------------------------------------- generator
+
+def test_generator_shapes_and_bf16_rounding():
+    w = ssd_inputs.workload("varlen32k", seqlen=4096, num_seqs=5)
+    inp = ssd_inputs.make_inputs(w)
+    assert inp["x"].shape == (1, 4096, 48, 64)
+    cu = inp["cu_seqlens"]
+    assert cu[0] == 0 and cu[-1] == 4096 and np.all(np.diff(cu) >= 64) and len(cu) == 6
+    for k in ("x", "dt", "B", "C"):
+        bits = inp[k].view(np.uint32)
+        assert np.all(bits & 0xFFFF == 0)
+    assert inp["initial_states"].shape == (5, 48, 64, 128)
+    # reproducible
+    again = ssd_inputs.make_inputs(w)
+    assert np.array_equal(again["x"], inp["x"]) and np.array_equal(again["cu_seqlens"], cu)
+
+
+def test_round_to_bf16_ties_to_even():
+    # 1 + 2^-8 is a tie between 1 and 1 + 2^-7: rounds to the even mantissa (1.0)
+    v = np.array([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -2.5], dtype=np.float32)
+    r = ssd_inputs.round_to_bf16(v)
+    assert r[0] == 1.0 and r[1] == 1.0 + 2.0 ** -6 and r[2] == -2.5
