@@ -1,0 +1,401 @@
+"""SSD forward benchmark (Mamba-2 SSD layer, forward pass) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload mamba2_2p7b] [--path auto|simt|tensor]
+
+One step = one ssd_fwd over the whole workload (every kernel of the path).
+Prints ONE JSON line on rank 0. For N > 1 (torchrun, one process per GPU)
+every rank runs its own copy of the workload (independent problems: weak
+scaling, no data-path collective); the step time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the slow, obviously-correct
+recurrence) on the host cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import signal
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import ssd_inputs  # noqa: E402
+
+L2_FLUSH_BYTES = 512 << 20        # > 4x the 126 MB L2
+FALLBACK_HBM_GBS = 6650.0
+THROTTLE_BITS = {
+    0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+    0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+    0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+}
+
+
+# --------------------------------------------------------------- accounting
+
+def algorithmic_bytes(inp: dict) -> int:
+    """Compulsory I/O of one forward: x, y, dt, B, C (+ initial / final states)."""
+    x, dt, B, C = inp["x"], inp["dt"], inp["B"], inp["C"]
+    es = 2 if inp["io_dtype"] == "bf16" else 4
+    n = (2 * x.size + dt.size + B.size + C.size) * es
+    H, P, N = x.shape[2], x.shape[3], B.shape[3]
+    nseq = inp["workload"].nseq
+    if inp.get("initial_states") is not None:
+        n += nseq * H * P * N * 4
+    if inp.get("want_final_states"):
+        n += nseq * H * P * N * 4
+    return int(n)
+
+
+def algorithmic_flops(inp: dict) -> int:
+    """Useful (causal-halved) FLOPs of the chunked algorithm per forward:
+    per token H * (4PN + Q*P) + G * Q * N."""
+    x, B = inp["x"], inp["B"]
+    tokens = x.shape[0] * x.shape[1]
+    H, P, G, N = x.shape[2], x.shape[3], B.shape[2], B.shape[3]
+    Q = inp["chunk_len"]
+    return int(tokens * (H * (4 * P * N + Q * P) + G * Q * N))
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "mamba_ssd_layer_fwd_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, fn), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def committed_traffic(workload: str, kernel: str):
+    """dram read+write bytes per launch from the committed ncu summary, if it
+    was taken on the current kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+        e = d[workload]
+        if e.get("kernel") == kernel and e.get("source_hash") == kernel_source_hash():
+            return int(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+    return None
+
+
+# ------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.path = None
+        self.gpu_index = gpu_index
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="clocks", suffix=".csv")
+            os.close(fd)
+            q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.gpu_index)], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.send_signal(signal.SIGTERM)
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 5:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), int(parts[4], 16)))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        reasons = set()
+        for _, _, bits in rows:
+            for b, name in THROTTLE_BITS.items():
+                if bits & b and name != "gpu_idle":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ------------------------------------------------------------ CPU baseline
+
+def cpu_oracle_rate(inp: dict, budget_s: float = 10.0):
+    """Time the fp64 oracle on the host cores on a bounded sample of
+    (sequence, head) pairs; returns (tokens/s scaled to the full workload,
+    cores, description)."""
+    import oracle
+    oracle.build()
+    cores = oracle.max_threads()
+    x = inp["x"]
+    H = x.shape[2]
+    bounds = ssd_inputs.seq_bounds(inp)
+    order = [(s, h) for h in range(H) for s in range(len(bounds))]
+    rng = np.random.default_rng(0)
+    order = [order[i] for i in rng.permutation(len(order))]
+    oracle.recurrence_pairs(inp, order[:1])             # warm (load, page in)
+    done_tok = 0
+    done_pairs = 0
+    t_total = 0.0
+    i = 0
+    batch = cores
+    while i < len(order) and t_total < budget_s:
+        pairs = order[i:i + batch]
+        t0 = time.perf_counter()
+        oracle.recurrence_pairs(inp, pairs, nthreads=cores)
+        dt = time.perf_counter() - t0
+        t_total += dt
+        done_tok += sum(bounds[s][1] for s, _ in pairs)
+        done_pairs += len(pairs)
+        i += len(pairs)
+        if dt > 0 and t_total < budget_s:
+            batch = max(cores, int(len(pairs) * min(4.0, (budget_s - t_total) / dt)))
+    token_heads_per_s = done_tok / t_total
+    desc = (f"{done_pairs} of {len(order)} (sequence, head) pairs ({done_tok} token-heads), "
+            f"random order, full sequence length; tokens/s = token-heads/s / {H} heads")
+    return token_heads_per_s / H, cores, desc, t_total
+
+
+# ------------------------------------------------------------------ helpers
+
+def make_workload(args):
+    w = ssd_inputs.workload(args.workload)
+    return ssd_inputs.make_inputs(w, seed=args.seed)
+
+
+def config_of(inp, args, n_gpus):
+    w = inp["workload"]
+    return {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "num_seqs": w.num_seqs,
+            "nheads": w.nheads, "headdim": w.headdim, "dstate": w.dstate, "ngroups": w.ngroups,
+            "chunk_len": inp["chunk_len"], "io_dtype": w.io_dtype,
+            "initial_states": bool(w.with_initial_states), "final_states": bool(w.with_final_states),
+            "tokens_per_gpu": w.tokens, "parallelism": f"replicas x{n_gpus}" if n_gpus > 1 else "1 gpu",
+            "l2": "flushed before every timed step (512 MiB write)", "path": args.path}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    inp = make_workload(args)
+    tokens = inp["x"].shape[0] * inp["x"].shape[1]
+    per_step = []
+    cores = 1
+    desc = ""
+    budget = max(1.0, min(args.ref_seconds, 150.0 / (args.warmup + args.steps)))
+    for i in range(args.warmup + args.steps):
+        rate, cores, desc, t = cpu_oracle_rate(inp, budget_s=budget)
+        if i >= args.warmup:
+            per_step.append(rate)
+    value = float(statistics.median(per_step))
+    line = {
+        "impl": "reference", "metric": "SSD fwd tokens/s", "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * tokens / value, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": config_of(inp, args, 1),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": "each step: " + desc},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import mamba_ssd_layer_fwd_b200 as ssd
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    inp = make_workload(args)
+    io = torch.bfloat16 if inp["io_dtype"] == "bf16" else torch.float32
+    host = {k: torch.from_numpy(inp[k]).to(io).pin_memory() for k in ("x", "dt", "B", "C")}
+    for k in ("A_log", "D", "initial_states"):
+        host[k] = None if inp[k] is None else torch.from_numpy(inp[k]).pin_memory()
+    host["cu_seqlens"] = None if inp["cu_seqlens"] is None else torch.from_numpy(inp["cu_seqlens"]).pin_memory()
+    d = {k: (None if v is None else v.to(dev)) for k, v in host.items()}
+    x = d["x"]
+    want_final = bool(inp["want_final_states"])
+    nseq = inp["workload"].nseq
+    H, P, N = x.shape[2], x.shape[3], d["B"].shape[3]
+    y = torch.empty_like(x)
+    fin = torch.empty((nseq, H, P, N), dtype=torch.float32, device=dev) if want_final else None
+    params = ssd.params_for(x, d["B"], inp["chunk_len"], d["cu_seqlens"], True, args.path)
+    ws = torch.empty(ssd.workspace_size(params), dtype=torch.uint8, device=dev)
+    launches_per_step = ssd.launch_count(params)
+    path = ssd.resolved_path(params)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(prof=None):
+        ssd.ssd_fwd(d["x"], d["dt"], d["A_log"], d["B"], d["C"], d["D"], chunk_len=inp["chunk_len"],
+                    initial_states=d["initial_states"], cu_seqlens=d["cu_seqlens"], y=y,
+                    final_states=fin, workspace=ws, stream=stream, path=args.path, prof_events=prof)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    rc = ssd.library().ssd_get_status(ws.data_ptr(), stream.cuda_stream or None)
+    if rc != 0:
+        raise ssd.SsdError(rc, "warm-up device status")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    for row in ev:              # torch creates events lazily: record once so the handles exist
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.current_device() if world == 1 else local)
+    if rank == 0:
+        sampler.start()
+        time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    for i in range(K):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step(prof=(ev[i][1], ev[i][2]))
+        ev[i][3].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    wall = time.perf_counter() - wall0
+    clocks = sampler.stop() if rank == 0 else None
+    step_ms = [ev[i][0].elapsed_time(ev[i][3]) for i in range(K)]
+    main_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+    ms = statistics.mean(step_ms)
+    kms = statistics.mean(main_ms)
+    if world > 1:
+        t = torch.tensor([ms, kms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, kms = float(t[0]), float(t[1])
+
+    # end to end: pinned host inputs -> device -> ssd_fwd -> result back to pinned host memory
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    fin_host = torch.empty(fin.shape, dtype=fin.dtype).pin_memory() if fin is not None else None
+    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+    d2h = y_host.numel() * y_host.element_size() + (fin_host.numel() * 4 if fin_host is not None else 0)
+    e2e_ms = []
+    for i in range(args.warmup + K):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        flush.zero_()
+        e0.record(stream)
+        for k, v in host.items():
+            if v is not None:
+                d[k].copy_(v, non_blocking=True)
+        step()
+        y_host.copy_(y, non_blocking=True)
+        if fin_host is not None:
+            fin_host.copy_(fin, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(e0.elapsed_time(e1))
+    e2e = statistics.mean(e2e_ms)
+    if world > 1:
+        t = torch.tensor([e2e], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e = float(t[0])
+
+    tokens = inp["x"].shape[0] * inp["x"].shape[1]
+    total_tokens = tokens * world
+    value = total_tokens / (ms * 1e-3)
+    alg_bytes = algorithmic_bytes(inp)
+    flops = algorithmic_flops(inp)
+    peak, peak_kind = measured_peaks()
+    kernel = "ssd_tc_walk" if path == "tensor" else "chunk_scan_kernel"
+    achieved = alg_bytes / (kms * 1e-3) / 1e9
+    line = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            rate, cores, desc, _ = cpu_oracle_rate(inp, budget_s=args.ref_seconds)
+            cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc}
+        line = {
+            "metric": "SSD fwd tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": inp["io_dtype"],
+            "data": "synthetic (seeded generator, value distributions of the workload)",
+            "config": config_of(inp, args, world),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": committed_traffic(args.workload, kernel),
+                         "kernel": kernel, "kernel_ms": kms, "alg_bytes": alg_bytes,
+                         "peak_source": f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"},
+            "tflops": flops / (ms * 1e-3) / 1e12,
+            "cpu_baseline": cpu,
+            "e2e": {"value": total_tokens / (e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches_per_step * K,
+            "clocks": clocks,
+            "path": path,
+            "wall_s_timed_region": wall,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mamba2_2p7b", choices=sorted(ssd_inputs.WORKLOADS))
+    ap.add_argument("--path", default="auto", choices=["auto", "simt", "tensor"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--ref-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)      # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

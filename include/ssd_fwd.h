@@ -1,0 +1,137 @@
+/*
+ * ssd_fwd.h - C ABI of the Mamba-2 SSD (structured state space duality)
+ * forward layer for NVIDIA B200 (sm_100a).
+ *
+ * The operation ("Transformers are SSMs: Generalized Models and Efficient
+ * Algorithms Through Structured State Space Duality", Sec. 2.4 "SSD layer",
+ * Sec. 3.4.1 eq. (8), Sec. 6 "SSD algorithm", Sec. 7.2 grouped heads,
+ * Sec. 8.3 variable length), per sequence s and head h, with B/C group
+ * g = h / (nheads / ngroups):
+ *
+ *     delta_t = softplus(dt[t, h])        (dt itself when dt_softplus == 0)
+ *     a_t     = exp(delta_t * A_h),  A_h = -exp(A_log[h])
+ *     state_t = a_t * state_{t-1} + (delta_t * x[t, h, :]) (outer) B[t, g, :]   (P x N, fp32)
+ *     y[t, h, :] = state_t @ C[t, g, :] + D[h] * x[t, h, :]
+ *
+ * with state_{-1} = initial_states[s, h] (zeros when NULL) and
+ * final_states[s, h] = the state after the sequence's last token.  It is
+ * evaluated by the chunked block decomposition of the semiseparable matrix
+ * M = L o (C B^T) (Sec. 6): quadratic form inside chunks, chunk states,
+ * a scan over chunk states, state-to-output.  The result does not depend on
+ * chunk_len except through rounding.
+ *
+ * Layouts (row-major, contiguous, every pointer 16-byte aligned):
+ *     x, y             (batch, seqlen, nheads, headdim)     io dtype
+ *     dt               (batch, seqlen, nheads)              io dtype
+ *     B, C             (batch, seqlen, ngroups, dstate)     io dtype
+ *     A_log, D         (nheads)                             float32
+ *     initial_states,
+ *     final_states     (nseq, nheads, headdim, dstate)      float32
+ *     cu_seqlens       (num_seqs + 1)                       int32
+ * nseq = num_seqs when cu_seqlens is given (packed variable-length batch:
+ * batch == 1, seqlen == total tokens, sequence i = tokens
+ * [cu_seqlens[i], cu_seqlens[i+1]) with no state crossing a boundary),
+ * else nseq = batch.
+ *
+ * Ownership and threading: every data pointer is a DEVICE pointer owned by
+ * the caller; the library allocates and frees nothing and keeps no mutable
+ * global state.  Calls are asynchronous on `stream` (a cudaStream_t passed as
+ * void*, NULL = legacy default stream); calls on different streams with
+ * different workspaces may run concurrently.
+ *
+ * Errors: arguments are validated on the host before anything is launched,
+ * and no C++ exception crosses this boundary.  Problems the host cannot see
+ * (a malformed cu_seqlens, a device-side wait that ran out of its bound) are
+ * recorded in the workspace's status word; read it with ssd_get_status().
+ */
+#ifndef SSD_FWD_H_
+#define SSD_FWD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SSD_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define SSD_API __attribute__((visibility("default")))
+#else
+#define SSD_API
+#endif
+
+typedef enum ssd_status {
+    SSD_OK = 0,
+    SSD_ERR_INVALID_ARG = -1,   /* null/misaligned pointer, bad dimension, workspace too small */
+    SSD_ERR_UNSUPPORTED = -2,   /* valid shape this build does not implement (see limits) */
+    SSD_ERR_CUDA = -3,          /* a CUDA runtime call or launch failed */
+    SSD_ERR_TIMEOUT = -4,       /* device-side bounded wait gave up (status word) */
+    SSD_ERR_BAD_SEQLENS = -5    /* cu_seqlens not 0 = c0 <= c1 <= ... = seqlen (status word) */
+} ssd_status;
+
+typedef enum ssd_dtype {
+    SSD_DTYPE_F32 = 0,          /* x, dt, B, C, y in float32 */
+    SSD_DTYPE_BF16 = 1          /* x, dt, B, C, y in bfloat16 (states stay float32) */
+} ssd_dtype;
+
+typedef enum ssd_path {
+    SSD_PATH_AUTO = 0,          /* tensor-core path when the shape allows it, else SIMT */
+    SSD_PATH_SIMT = 1,          /* CUDA-core path: any supported shape, float32 or bf16 */
+    SSD_PATH_TENSOR = 2         /* tcgen05/TMEM path: bf16, headdim 64, dstate 64/128/256 */
+} ssd_path;
+
+typedef struct ssd_fwd_params {
+    int batch;                  /* >= 1 (1 when num_seqs > 0) */
+    int seqlen;                 /* >= 0, tokens per row (total tokens when num_seqs > 0) */
+    int nheads;                 /* H >= 1 */
+    int headdim;                /* P: 1..128 (tensor path: 64) */
+    int dstate;                 /* N: 1..256 (tensor path: 64, 128 or 256) */
+    int ngroups;                /* G >= 1, nheads % ngroups == 0 */
+    int chunk_len;              /* Q: 64, 128 or 256 */
+    int num_seqs;               /* > 0 iff cu_seqlens != NULL */
+    ssd_dtype io_dtype;
+    int dt_softplus;            /* 1: delta = softplus(dt); 0: delta = dt (must be >= 0) */
+    ssd_path path;
+    void *prof_begin;           /* optional cudaEvent_t recorded on `stream` right before the main kernel */
+    void *prof_end;             /* optional cudaEvent_t recorded right after it */
+} ssd_fwd_params;
+
+/* Bytes of device workspace ssd_fwd needs for these parameters (0 on invalid
+ * parameters).  The workspace must be 256-byte aligned; its contents need no
+ * initialisation and may be reused by the next call on the same stream. */
+SSD_API size_t ssd_fwd_workspace_size(const ssd_fwd_params *p);
+
+/* SSD forward.  D, initial_states, cu_seqlens and final_states may be NULL
+ * (D = 0, zero initial state, batch of equal rows, no final state written).
+ * Returns SSD_OK once every kernel is enqueued; see ssd_get_status for the
+ * device-side outcome. */
+SSD_API ssd_status ssd_fwd(const ssd_fwd_params *p,
+                   const void *x, const void *dt, const float *A_log,
+                   const void *B, const void *C, const float *D,
+                   const float *initial_states, const int32_t *cu_seqlens,
+                   void *y, float *final_states,
+                   void *workspace, size_t workspace_bytes, void *stream);
+
+/* Device-side status of the last ssd_fwd that used `workspace` on `stream`:
+ * synchronises `stream`, then returns SSD_OK, SSD_ERR_TIMEOUT or
+ * SSD_ERR_BAD_SEQLENS (or SSD_ERR_CUDA if the copy fails). */
+SSD_API ssd_status ssd_get_status(const void *workspace, void *stream);
+
+/* Number of kernels one ssd_fwd call with these parameters launches. */
+SSD_API int ssd_fwd_launch_count(const ssd_fwd_params *p);
+
+/* The path ssd_fwd takes for these parameters (AUTO resolved), or -1. */
+SSD_API int ssd_fwd_resolved_path(const ssd_fwd_params *p);
+
+/* Static description of a status code. */
+SSD_API const char *ssd_status_string(ssd_status s);
+
+SSD_API int ssd_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSD_FWD_H_ */

@@ -1,0 +1,205 @@
+"""Mamba-2 SSD forward layer for NVIDIA B200 (sm_100a): Python binding.
+
+A thin ctypes layer over the C ABI in include/ssd_fwd.h (libssd_b200.so).
+It only marshals arguments: PyTorch provides device memory and the stream,
+every step of the computation runs in the library's CUDA kernels. There is no
+CPU fallback; calling without the built library raises.
+
+    import torch, mamba_ssd_layer_fwd_b200 as ssd
+    y, final = ssd.ssd_fwd(x, dt, A_log, B, C, D, chunk_len=256,
+                           return_final_states=True)
+
+Shapes (contiguous): x (batch, seqlen, nheads, headdim), dt (batch, seqlen,
+nheads), B and C (batch, seqlen, ngroups, dstate), A_log and D (nheads,)
+float32, initial_states (nseq, nheads, headdim, dstate) float32, cu_seqlens
+(nseq + 1,) int32 for a packed batch (batch == 1).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+__all__ = [
+    "ssd_fwd", "SsdParams", "workspace_size", "launch_count", "resolved_path", "library",
+    "library_path", "STATUS", "PATHS", "SsdError",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "_lib", "libssd_b200.so")
+_lib = None
+_lock = threading.Lock()
+
+STATUS = {0: "SSD_OK", -1: "SSD_ERR_INVALID_ARG", -2: "SSD_ERR_UNSUPPORTED", -3: "SSD_ERR_CUDA",
+          -4: "SSD_ERR_TIMEOUT", -5: "SSD_ERR_BAD_SEQLENS"}
+PATHS = {"auto": 0, "simt": 1, "tensor": 2}
+DTYPES = {"f32": 0, "bf16": 1}
+
+EXPORTED = ("ssd_fwd", "ssd_fwd_workspace_size", "ssd_get_status", "ssd_fwd_launch_count",
+            "ssd_fwd_resolved_path", "ssd_status_string", "ssd_abi_version")
+
+
+class SsdError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {STATUS.get(code, code)} ({_status_string(code)})")
+
+
+class SsdParams(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int), ("seqlen", ctypes.c_int), ("nheads", ctypes.c_int),
+        ("headdim", ctypes.c_int), ("dstate", ctypes.c_int), ("ngroups", ctypes.c_int),
+        ("chunk_len", ctypes.c_int), ("num_seqs", ctypes.c_int), ("io_dtype", ctypes.c_int),
+        ("dt_softplus", ctypes.c_int), ("path", ctypes.c_int),
+        ("prof_begin", ctypes.c_void_p), ("prof_end", ctypes.c_void_p),
+    ]
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def library():
+    """Load libssd_b200.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                                   "`python -m mamba_ssd_layer_fwd_b200.build`")
+            lib = ctypes.CDLL(_LIB_PATH)
+            vp, sz, i32, pp = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.POINTER(SsdParams)
+            lib.ssd_fwd.restype = i32
+            lib.ssd_fwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+            lib.ssd_fwd_workspace_size.restype = sz
+            lib.ssd_fwd_workspace_size.argtypes = [pp]
+            lib.ssd_get_status.restype = i32
+            lib.ssd_get_status.argtypes = [vp, vp]
+            lib.ssd_fwd_launch_count.restype = i32
+            lib.ssd_fwd_launch_count.argtypes = [pp]
+            lib.ssd_fwd_resolved_path.restype = i32
+            lib.ssd_fwd_resolved_path.argtypes = [pp]
+            lib.ssd_status_string.restype = ctypes.c_char_p
+            lib.ssd_status_string.argtypes = [i32]
+            lib.ssd_abi_version.restype = i32
+            lib.ssd_abi_version.argtypes = []
+            _lib = lib
+    return _lib
+
+
+def _status_string(code: int) -> str:
+    try:
+        return library().ssd_status_string(int(code)).decode()
+    except Exception:  # library missing: keep the error message usable
+        return "?"
+
+
+def make_params(*, batch, seqlen, nheads, headdim, dstate, ngroups, chunk_len, num_seqs=0,
+                io_dtype="bf16", dt_softplus=True, path="auto", prof_begin=None,
+                prof_end=None) -> SsdParams:
+    return SsdParams(int(batch), int(seqlen), int(nheads), int(headdim), int(dstate), int(ngroups),
+                     int(chunk_len), int(num_seqs), DTYPES[io_dtype], int(bool(dt_softplus)),
+                     PATHS[path], prof_begin, prof_end)
+
+
+def workspace_size(params: SsdParams) -> int:
+    return int(library().ssd_fwd_workspace_size(ctypes.byref(params)))
+
+
+def launch_count(params: SsdParams) -> int:
+    return int(library().ssd_fwd_launch_count(ctypes.byref(params)))
+
+
+def resolved_path(params: SsdParams) -> str:
+    r = int(library().ssd_fwd_resolved_path(ctypes.byref(params)))
+    return {1: "simt", 2: "tensor"}.get(r, "unsupported")
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else int(t.data_ptr())
+
+
+def _stream_handle(stream) -> Optional[int]:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) or None
+
+
+def params_for(x, B, chunk_len: int, cu_seqlens=None, dt_softplus=True, path="auto",
+               prof_events=None) -> SsdParams:
+    import torch
+    if x.dtype == torch.bfloat16:
+        io = "bf16"
+    elif x.dtype == torch.float32:
+        io = "f32"
+    else:
+        raise TypeError(f"x must be bfloat16 or float32, got {x.dtype}")
+    b, T, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    nseq = 0 if cu_seqlens is None else int(cu_seqlens.numel()) - 1
+    pb = pe = None
+    if prof_events is not None:
+        pb, pe = (int(e.cuda_event) for e in prof_events)
+    return make_params(batch=b, seqlen=T, nheads=H, headdim=P, dstate=N, ngroups=G,
+                       chunk_len=chunk_len, num_seqs=nseq, io_dtype=io, dt_softplus=dt_softplus,
+                       path=path, prof_begin=pb, prof_end=pe)
+
+
+def ssd_fwd(x, dt, A_log, B, C, D=None, chunk_len: int = 256, initial_states=None,
+            cu_seqlens=None, dt_softplus: bool = True, return_final_states: bool = False,
+            y=None, final_states=None, workspace=None, stream=None, path: str = "auto",
+            prof_events=None, check_status: bool = False):
+    """SSD forward on the GPU through the C ABI. Returns y, or (y, final_states)
+    when `return_final_states` is true (or `final_states` is given).
+
+    x, dt, B, C share the io dtype (bfloat16 or float32); A_log, D,
+    initial_states are float32; cu_seqlens is int32. Outputs and the workspace
+    are allocated with torch on x's device unless passed in. `prof_events` =
+    (begin, end) torch.cuda.Event pair recorded around the main kernel.
+    """
+    import torch
+    lib = library()
+    dev = x.device
+    if dev.type != "cuda":
+        raise ValueError("ssd_fwd runs on CUDA tensors only")
+    for name, t in (("x", x), ("dt", dt), ("B", B), ("C", C)):
+        if t.dtype != x.dtype or not t.is_contiguous() or t.device != dev:
+            raise ValueError(f"{name} must be a contiguous {x.dtype} tensor on {dev}")
+    for name, t in (("A_log", A_log), ("D", D), ("initial_states", initial_states)):
+        if t is not None and (t.dtype != torch.float32 or not t.is_contiguous() or t.device != dev):
+            raise ValueError(f"{name} must be a contiguous float32 tensor on {dev}")
+    if cu_seqlens is not None and (cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_contiguous()):
+        raise ValueError("cu_seqlens must be a contiguous int32 tensor")
+    if x.dim() != 4 or dt.shape != x.shape[:3] or B.shape != C.shape or B.shape[:2] != x.shape[:2]:
+        raise ValueError("shape mismatch between x, dt, B, C")
+    p = params_for(x, B, chunk_len, cu_seqlens, dt_softplus, path, prof_events)
+    b, T, H, P = x.shape
+    N = B.shape[3]
+    nseq = p.num_seqs if p.num_seqs > 0 else b
+    if y is None:
+        y = torch.empty_like(x)
+    want_final = return_final_states or final_states is not None
+    if want_final and final_states is None:
+        final_states = torch.empty((nseq, H, P, N), dtype=torch.float32, device=dev)
+    if initial_states is not None and tuple(initial_states.shape) != (nseq, H, P, N):
+        raise ValueError(f"initial_states must have shape {(nseq, H, P, N)}")
+    if final_states is not None and tuple(final_states.shape) != (nseq, H, P, N):
+        raise ValueError(f"final_states must have shape {(nseq, H, P, N)}")
+    need = int(lib.ssd_fwd_workspace_size(ctypes.byref(p)))
+    if need == 0:
+        raise SsdError(-2 if lib.ssd_fwd_resolved_path(ctypes.byref(p)) == -1 else -1, "ssd_fwd_workspace_size")
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    st = _stream_handle(stream)
+    rc = lib.ssd_fwd(ctypes.byref(p), _ptr(x), _ptr(dt), _ptr(A_log), _ptr(B), _ptr(C), _ptr(D),
+                     _ptr(initial_states), _ptr(cu_seqlens), _ptr(y), _ptr(final_states),
+                     _ptr(workspace), workspace.numel() * workspace.element_size(), st)
+    if rc != 0:
+        raise SsdError(rc, "ssd_fwd")
+    if check_status:
+        rc = lib.ssd_get_status(_ptr(workspace), st)
+        if rc != 0:
+            raise SsdError(rc, "ssd_fwd (device status)")
+    return (y, final_states) if want_final else y

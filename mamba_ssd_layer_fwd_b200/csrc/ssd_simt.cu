@@ -1,0 +1,333 @@
+// CUDA-core (SIMT) path of the SSD forward: the chunked block decomposition
+// of "Transformers are SSMs", Sec. 6, as four kernels with fp32 arithmetic.
+// It serves float32 inputs (where bf16 tensor-core operands would not meet a
+// 1e-4 tolerance) and every shape the tensor-core path does not take.
+//
+//   chunk_cumsum   delta = softplus(dt), dA = delta * A, inclusive prefix
+//                  sum of dA inside each chunk (the 1-SS mask's exponents,
+//                  Sec. 3.2.2 / Listing 1 `segsum`)
+//   chunk_state    S_c = sum_l exp(cs_last - cs_l) delta_l x_l (outer) B_l:
+//                  the chunk's final state from a zero start (Sec. 6.2,
+//                  right factor)
+//   state_passing  H_c = exp(cs_last(c-1)) H_{c-1} + S_{c-1}, H_0 = initial
+//                  state: the state entering every chunk (Sec. 6.2, centre
+//                  factor, evaluated as the sequential scalar scan of App. B)
+//   chunk_scan     y_l = sum_{s<=l} (C_l . B_s) exp(cs_l - cs_s) delta_s x_s
+//                        + exp(cs_l) C_l . H_c + D x_l
+//                  (Sec. 6.1 diagonal block + Sec. 6.2 left factor)
+#include "ssd_common.cuh"
+
+namespace ssd {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kTile = 32;   // rows per smem tile
+
+// ------------------------------------------------------------------ cumsum
+template <typename T>
+__global__ void __launch_bounds__(256)
+chunk_cumsum_kernel(Plan plan, Dims d, const T *__restrict__ dt, const float *__restrict__ A_log,
+                    float *__restrict__ cs, float *__restrict__ dv)
+{
+    __shared__ float s_warp[8];
+    const int c = blockIdx.x;
+    if (c >= *plan.count) return;
+    const ChunkDesc ch = plan.chunks[c];
+    const int h = blockIdx.y;
+    const int l = threadIdx.x;          // blockDim.x == Q
+    const float A = -expf(A_log[h]);
+    float delta = 0.0f, dA = 0.0f;
+    if (l < ch.len) {
+        const float r = to_f32(dt[(size_t)(ch.tok0 + l) * d.H + h]);
+        delta = d.dt_softplus ? fmaxf(r, 0.0f) + log1pf(expf(-fabsf(r))) : r;
+        dA = delta * A;
+    }
+    // inclusive scan over the chunk
+    float v = dA;
+    for (int o = 1; o < 32; o <<= 1) {
+        const float u = __shfl_up_sync(0xffffffffu, v, o);
+        if ((l & 31) >= o) v += u;
+    }
+    if ((l & 31) == 31) s_warp[l >> 5] = v;
+    __syncthreads();
+    float carry = 0.0f;
+    for (int w = 0; w < (l >> 5); ++w) carry += s_warp[w];
+    const size_t o = ((size_t)c * d.H + h) * d.Q + l;
+    cs[o] = v + carry;
+    dv[o] = delta;
+}
+
+// -------------------------------------------------------------- chunk_state
+constexpr int kStateEPT = 16;   // outputs per thread per pass
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+chunk_state_kernel(Plan plan, Dims d, const T *__restrict__ x, const T *__restrict__ Bm,
+                   const float *__restrict__ cs, const float *__restrict__ dv,
+                   float *__restrict__ states)
+{
+    extern __shared__ float smem[];
+    const int c = blockIdx.x;
+    if (c >= *plan.count) return;
+    const ChunkDesc ch = plan.chunks[c];
+    const int h = blockIdx.y;
+    const int g = h / d.heads_per_group;
+    const int P = d.P, N = d.N, Q = d.Q;
+    float *Xs = smem;                       // kTile x P   (weighted x)
+    float *Bs = Xs + kTile * P;             // kTile x N
+    float *w = Bs + kTile * N;              // Q
+    const float *csc = cs + ((size_t)c * d.H + h) * Q;
+    const float *dvc = dv + ((size_t)c * d.H + h) * Q;
+    const float cs_last = csc[Q - 1];
+    for (int l = threadIdx.x; l < Q; l += kThreads)
+        w[l] = l < ch.len ? __expf(cs_last - csc[l]) * dvc[l] : 0.0f;
+    __syncthreads();
+
+    const int PN = P * N;
+    float *out = states + ((size_t)c * d.H + h) * PN;
+    for (int e0 = 0; e0 < PN; e0 += kThreads * kStateEPT) {
+        float acc[kStateEPT];
+#pragma unroll
+        for (int i = 0; i < kStateEPT; ++i) acc[i] = 0.0f;
+        for (int l0 = 0; l0 < ch.len; l0 += kTile) {
+            for (int i = threadIdx.x; i < kTile * P; i += kThreads) {
+                const int r = i / P, p = i % P;
+                const int l = l0 + r;
+                Xs[i] = l < ch.len ? w[l] * to_f32(x[((size_t)(ch.tok0 + l) * d.H + h) * P + p]) : 0.0f;
+            }
+            for (int i = threadIdx.x; i < kTile * N; i += kThreads) {
+                const int r = i / N, n = i % N;
+                const int l = l0 + r;
+                Bs[i] = l < ch.len ? to_f32(Bm[((size_t)(ch.tok0 + l) * d.G + g) * N + n]) : 0.0f;
+            }
+            __syncthreads();
+#pragma unroll
+            for (int i = 0; i < kStateEPT; ++i) {
+                const int e = e0 + threadIdx.x + i * kThreads;
+                if (e < PN) {
+                    const int p = e / N, n = e % N;
+                    float a = acc[i];
+                    for (int j = 0; j < kTile; ++j) a = fmaf(Xs[j * P + p], Bs[j * N + n], a);
+                    acc[i] = a;
+                }
+            }
+            __syncthreads();
+        }
+#pragma unroll
+        for (int i = 0; i < kStateEPT; ++i) {
+            const int e = e0 + threadIdx.x + i * kThreads;
+            if (e < PN) out[e] = acc[i];
+        }
+    }
+}
+
+// ------------------------------------------------------------ state_passing
+__global__ void __launch_bounds__(kThreads)
+state_passing_kernel(Plan plan, Dims d, const float *__restrict__ cs, float *__restrict__ states,
+                     const float *__restrict__ init, float *__restrict__ final_states)
+{
+    const int s = blockIdx.x;
+    const int h = blockIdx.y;
+    const int PN = d.P * d.N;
+    const int e = blockIdx.z * kThreads + threadIdx.x;
+    if (e >= PN) return;
+    const SeqDesc sq = plan.seqs[s];
+    float hv = init ? init[((size_t)s * d.H + h) * PN + e] : 0.0f;
+    for (int j = 0; j < sq.nchunks; ++j) {
+        const int c = sq.chunk0 + j;
+        const size_t idx = ((size_t)c * d.H + h) * PN + e;
+        const float sv = states[idx];
+        states[idx] = hv;                       // state entering chunk c
+        const float decay = __expf(cs[((size_t)c * d.H + h) * d.Q + d.Q - 1]);
+        hv = fmaf(decay, hv, sv);
+    }
+    if (final_states) final_states[((size_t)s * d.H + h) * PN + e] = hv;
+}
+
+// --------------------------------------------------------------- chunk_scan
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+chunk_scan_kernel(Plan plan, Dims d, const T *__restrict__ x, const T *__restrict__ Bm,
+                  const T *__restrict__ Cm, const float *__restrict__ D,
+                  const float *__restrict__ cs, const float *__restrict__ dv,
+                  const float *__restrict__ states, T *__restrict__ y)
+{
+    extern __shared__ float smem[];
+    const int c = blockIdx.x;
+    if (c >= *plan.count) return;
+    const ChunkDesc ch = plan.chunks[c];
+    const int l0 = blockIdx.z * kTile;
+    if (l0 >= ch.len) return;
+    const int h = blockIdx.y;
+    const int g = h / d.heads_per_group;
+    const int P = d.P, N = d.N, Q = d.Q;
+    const int NS = N + 1, PS = P + 1;       // padded strides
+    float *Cs = smem;                       // kTile x NS
+    float *Bs = Cs + kTile * NS;            // kTile x NS
+    float *Xs = Bs + kTile * NS;            // kTile x PS
+    float *Hs = Xs + kTile * PS;            // kTile x PS  (32 state rows n, all p)
+    float *Gm = Hs + kTile * PS;            // kTile x (kTile + 1)
+    float *csl = Gm + kTile * (kTile + 1);  // kTile
+    float *css = csl + kTile;               // kTile
+    float *dvs = css + kTile;               // kTile
+    const float *csc = cs + ((size_t)c * d.H + h) * Q;
+    const float *dvc = dv + ((size_t)c * d.H + h) * Q;
+    const float *Hc = states + ((size_t)c * d.H + h) * (size_t)P * N;   // state entering chunk
+
+    for (int i = threadIdx.x; i < kTile * N; i += kThreads) {
+        const int r = i / N, n = i % N;
+        const int l = l0 + r;
+        Cs[r * NS + n] = l < ch.len ? to_f32(Cm[((size_t)(ch.tok0 + l) * d.G + g) * N + n]) : 0.0f;
+    }
+    if (threadIdx.x < kTile) csl[threadIdx.x] = csc[min(l0 + (int)threadIdx.x, Q - 1)];
+    __syncthreads();
+
+    // this thread's outputs: e = threadIdx.x + i * kThreads over kTile x P
+    constexpr int kMaxEPT = kTile * 128 / kThreads;  // P <= 128
+    float acc[kMaxEPT];
+#pragma unroll
+    for (int i = 0; i < kMaxEPT; ++i) acc[i] = 0.0f;
+    const int nout = kTile * P;
+
+    // left factor: exp(cs_l) * sum_n C[l][n] H[p][n], over n tiles of kTile
+    for (int n0 = 0; n0 < N; n0 += kTile) {
+        for (int i = threadIdx.x; i < kTile * P; i += kThreads) {
+            const int p = i / kTile, nn = i % kTile;
+            const int n = n0 + nn;
+            Hs[nn * PS + p] = n < N ? Hc[(size_t)p * N + n] : 0.0f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < kMaxEPT; ++i) {
+            const int e = threadIdx.x + i * kThreads;
+            if (e < nout) {
+                const int r = e / P, p = e % P;
+                float a = acc[i];
+                const int nmax = min(kTile, N - n0);
+                for (int nn = 0; nn < nmax; ++nn) a = fmaf(Cs[r * NS + n0 + nn], Hs[nn * PS + p], a);
+                acc[i] = a;
+            }
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < kMaxEPT; ++i) {
+        const int e = threadIdx.x + i * kThreads;
+        if (e < nout) acc[i] *= __expf(csl[e / P]);
+    }
+
+    // diagonal block: sum over s <= l of (C_l . B_s) exp(cs_l - cs_s) delta_s x_s
+    for (int s0 = 0; s0 <= l0; s0 += kTile) {
+        for (int i = threadIdx.x; i < kTile * N; i += kThreads) {
+            const int r = i / N, n = i % N;
+            const int s = s0 + r;
+            Bs[r * NS + n] = s < ch.len ? to_f32(Bm[((size_t)(ch.tok0 + s) * d.G + g) * N + n]) : 0.0f;
+        }
+        for (int i = threadIdx.x; i < kTile * P; i += kThreads) {
+            const int r = i / P, p = i % P;
+            const int s = s0 + r;
+            Xs[r * PS + p] = s < ch.len ? to_f32(x[((size_t)(ch.tok0 + s) * d.H + h) * P + p]) : 0.0f;
+        }
+        if (threadIdx.x < kTile) {
+            const int s = s0 + threadIdx.x;
+            css[threadIdx.x] = csc[min(s, Q - 1)];
+            dvs[threadIdx.x] = s < ch.len ? dvc[s] : 0.0f;
+        }
+        __syncthreads();
+        for (int i = threadIdx.x; i < kTile * kTile; i += kThreads) {
+            const int r = i / kTile, j = i % kTile;
+            const int l = l0 + r, s = s0 + j;
+            float v = 0.0f;
+            if (s <= l && s < ch.len) {
+                float dot = 0.0f;
+                for (int n = 0; n < N; ++n) dot = fmaf(Cs[r * NS + n], Bs[j * NS + n], dot);
+                v = dot * __expf(csl[r] - css[j]) * dvs[j];
+            }
+            Gm[r * (kTile + 1) + j] = v;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < kMaxEPT; ++i) {
+            const int e = threadIdx.x + i * kThreads;
+            if (e < nout) {
+                const int r = e / P, p = e % P;
+                float a = acc[i];
+                for (int j = 0; j < kTile; ++j) a = fmaf(Gm[r * (kTile + 1) + j], Xs[j * PS + p], a);
+                acc[i] = a;
+            }
+        }
+        __syncthreads();
+    }
+
+    const float Dh = D ? D[h] : 0.0f;
+#pragma unroll
+    for (int i = 0; i < kMaxEPT; ++i) {
+        const int e = threadIdx.x + i * kThreads;
+        if (e < nout) {
+            const int r = e / P, p = e % P;
+            const int l = l0 + r;
+            if (l < ch.len) {
+                const size_t o = ((size_t)(ch.tok0 + l) * d.H + h) * P + p;
+                y[o] = from_f32<T>(acc[i] + Dh * to_f32(x[o]));
+            }
+        }
+    }
+}
+
+size_t state_smem(const Dims &d) { return sizeof(float) * (kTile * d.P + kTile * d.N + d.Q); }
+size_t scan_smem(const Dims &d)
+{
+    return sizeof(float) * (2 * kTile * (d.N + 1) + 2 * kTile * (d.P + 1) + kTile * (kTile + 1) + 3 * kTile);
+}
+
+template <typename T>
+cudaError_t launch_typed(const Plan &plan, const Dims &d, const SimtArgs &a, cudaStream_t st,
+                         cudaEvent_t pb, cudaEvent_t pe)
+{
+    const T *x = static_cast<const T *>(a.x);
+    const T *dt = static_cast<const T *>(a.dt);
+    const T *Bm = static_cast<const T *>(a.B);
+    const T *Cm = static_cast<const T *>(a.C);
+    T *y = static_cast<T *>(a.y);
+    const dim3 gc(plan.max_chunks, d.H);
+    chunk_cumsum_kernel<T><<<gc, d.Q, 0, st>>>(plan, d, dt, a.A_log, a.cs, a.dv);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+
+    const size_t ss = state_smem(d);
+    e = cudaFuncSetAttribute(chunk_state_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ss);
+    if (e != cudaSuccess) return e;
+    chunk_state_kernel<T><<<gc, kThreads, ss, st>>>(plan, d, x, Bm, a.cs, a.dv, a.states);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    const dim3 gp(plan.nseq, d.H, (d.P * d.N + kThreads - 1) / kThreads);
+    state_passing_kernel<<<gp, kThreads, 0, st>>>(plan, d, a.cs, a.states, a.init, a.final_states);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    const size_t sc = scan_smem(d);
+    e = cudaFuncSetAttribute(chunk_scan_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sc);
+    if (e != cudaSuccess) return e;
+    const dim3 gs(plan.max_chunks, d.H, (d.Q + kTile - 1) / kTile);
+    if (pb) cudaEventRecord(pb, st);
+    chunk_scan_kernel<T><<<gs, kThreads, sc, st>>>(plan, d, x, Bm, Cm, a.D, a.cs, a.dv, a.states, y);
+    if (pe) cudaEventRecord(pe, st);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_simt(const Plan &plan, const Dims &d, const SimtArgs &a, cudaStream_t stream,
+                        cudaEvent_t prof_begin, cudaEvent_t prof_end)
+{
+    if (plan.max_chunks == 0) {
+        // nothing to compute; final states still equal the initial states
+        const dim3 gp(plan.nseq, d.H, (d.P * d.N + kThreads - 1) / kThreads);
+        if (a.final_states && plan.nseq > 0)
+            state_passing_kernel<<<gp, kThreads, 0, stream>>>(plan, d, a.cs, a.states, a.init, a.final_states);
+        return cudaGetLastError();
+    }
+    return a.bf16 ? launch_typed<__nv_bfloat16>(plan, d, a, stream, prof_begin, prof_end)
+                  : launch_typed<float>(plan, d, a, stream, prof_begin, prof_end);
+}
+
+}  // namespace ssd

@@ -1,0 +1,1041 @@
+// Tensor-core path of the SSD forward for sm_100a (tcgen05 / TMEM / TMA).
+//
+// Method ("Transformers are SSMs", Sec. 6, block decomposition of the
+// semiseparable matrix M = L o (C B^T)), evaluated by one CTA per work item
+// = (sequence, block of KH heads sharing a B/C group, token segment).  The
+// CTA walks its segment in 128-token blocks, keeping every head's P x N
+// state in tensor memory (fp32) between blocks, so chunk states never go
+// through HBM.  Per block c and head h (q = 128 tokens, rows l, columns s):
+//
+//   cs_l   = sum_{k<=l} delta_k A_h                     (cumsum warp, fp32)
+//   CB     = C_c B_c^T                    (UMMA, K = N; once per block, shared by the KH heads)
+//   Pm     = CB o exp(cs_l - cs_s) delta_s  (s <= l), + D_h on the diagonal
+//                                          (mask warps, TMEM -> regs -> TMEM as bf16)
+//   Yd     = Pm X_c                       (UMMA, A operand from TMEM)  Sec. 6.1
+//   Yo     = C_c Hbf^T,  Hbf = bf16(H)    (UMMA)                       Sec. 6.2 left factor
+//   y_l    = Yd_l + exp(cs_l) Yo_l        (epilogue warps -> HBM)
+//   H     <- exp(cs_last) H + B_c^T (w o X_c),  w_s = exp(cs_last - cs_s) delta_s
+//                                          (state warps rescale H in TMEM, UMMA accumulates)
+//                                          Sec. 6.2 right + centre factors
+//
+// Each diagonal block of the caller's chunk length Q (128 or 256) is thereby
+// computed by the same decomposition one level down with 128-token blocks;
+// Sec. 6.1 leaves the method for a diagonal block free, and the result is
+// the same up to rounding.
+//
+// Warp roles (16 warps; warp w runs on SM sub-partition w % 4 and may only
+// touch TMEM lanes 32*(w%4) .. +31): 0 cumsum, 1 UMMA issuer for the state
+// path (H += B^T (w o X)), 2 TMA producer, 3 UMMA issuer for the output
+// path (CB, C Hbf^T, Pm X) + TMEM owner, 4-7 and 10-11 mask (the causal
+// work of rows 96-127 is four times that of rows 0-31, so sub-partitions
+// 0-1 also get the w o X pass, warps 8-9), 12-15 state rescale + output
+// epilogue.  Two issuers keep the state and output paths from waiting on
+// each other.  Every mbarrier wait is bounded (2 s); on a timeout the CTA
+// records SSD_ERR_TIMEOUT in the status word, drains, frees TMEM and exits.
+//
+// When there are too few (sequence, head block) pairs to fill the GPU, each
+// sequence is cut into segments.  A first launch of the same kernel in
+// state-only mode computes every non-final segment's end state from zero;
+// a scan kernel turns those into each segment's entering state; the full
+// walk then starts every segment from its true state (Sec. 8.2: state
+// passing between pieces of a sequence).
+#include <cudaTypedefs.h>
+
+#include "ssd_tc.cuh"
+#include "ssd_tc_prims.cuh"
+
+namespace ssd {
+namespace {
+
+using namespace tc;
+
+constexpr int kQ = 128;          // tokens per block (TMEM lanes, UMMA M)
+constexpr int kP = 64;           // head dim
+constexpr int kThreadsTc = 512;  // 16 warps
+constexpr int kMaskWarps = 6;    // warps 4-7, 10, 11
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kCsd = 4;          // depth of the per-(block, head) cumsum ring
+constexpr int kPrefetch = 3;     // blocks of L2 prefetch ahead of the TMA loads
+
+struct TcItem {
+    int seq;     // sequence index
+    int tok0;    // first token of the segment (flattened token axis)
+    int len;     // tokens in the segment (>= 1)
+    int gseg;    // global segment index (segment-state buffer row)
+    int seg;     // segment index inside the sequence
+    int nseg;    // segments of the sequence
+    int h0;      // first head of the block
+    int pad;
+};
+
+struct TcParams {
+    const __nv_bfloat16 *dt;
+    const float *A_log, *D, *init;
+    __nv_bfloat16 *y;
+    float *final_states;
+    float *segstate;      // [max_segments][H][P][N]: pass-1 end states, then entering states
+    float *seglogdec;     // [max_segments][H]: sum of delta*A over the segment
+    const TcItem *items;
+    const int *count;
+    int *status;
+    int H, G, N, heads_per_group;
+    int dt_softplus;
+};
+
+// --------------------------------------------------------------- smem layout
+template <int NST>
+struct __align__(1024) TcSmem {
+    static constexpr int kBoxes = NST / 64;
+    uint8_t bc[2][2][kBoxes][16384];   // [stage][0 = C, 1 = B][64-column box][128 rows x 128 B]
+    uint8_t x[2][16384];               // X blocks (ring over (block, head))
+    uint8_t xw[2][16384];              // w o X (ring over (block, head))
+    uint8_t hbf[NST * 128];            // bf16(H)^T: rows n, 64 p per 128 B row
+    float cs2[kCsd][kQ];               // log2-scaled inclusive cumsum of delta*A
+    float dl[kCsd][kQ];                // delta_s (0 on padding rows)
+    float w[kCsd][kQ];                 // exp(cs_last - cs_s) * delta_s
+    float e[kCsd][kQ];                 // exp(cs_l)
+    float alpha[kCsd];                 // exp(cs_last)
+    float ldec[kCsd];                  // cs_last (natural log of the block decay)
+    uint64_t bc_full[2], bc_empty[2], x_full[2], x_empty[2], cs_full[kCsd], cs_empty[kCsd];
+    uint64_t cb_full, cb_empty, pm_full[2], pm_empty[2], hb_full, hb_empty, xw_full[2], xw_empty[2];
+    uint64_t h_ready[2], hs_full[2], y_full, yo_empty, yd_empty, drain_o, drain_s;
+    uint32_t tmem_base;
+    int abort;
+};
+
+template <int NST>
+constexpr size_t tc_smem_bytes()
+{
+    return sizeof(TcSmem<NST>) + 1024;   // + alignment slack
+}
+
+__device__ __forceinline__ void record_timeout(int *status) { set_status(status, kDevTimeout); }
+
+// TMEM column map
+constexpr uint32_t kColCB = 0, kColPm = 128, kColH = 256, kColYd = 384, kColYo = 448;
+
+// Optional per-CTA event timeline (SM clock), compiled only with -DSSD_TRACE.
+#ifdef SSD_TRACE
+constexpr int kTraceEvents = 28, kTraceUnits = 64, kTraceCtas = 8;
+__device__ long long *g_trace = nullptr;
+#define SSD_TRACE_EV(ev, idx)                                                                           \
+    do {                                                                                                \
+        if (trace_buf && (idx) < kTraceUnits)                                                           \
+            trace_buf[((size_t)blockIdx.x * kTraceEvents + (ev)) * kTraceUnits + (idx)] = clock64() - t_start; \
+    } while (0)
+#else
+#define SSD_TRACE_EV(ev, idx) \
+    do {                      \
+    } while (0)
+#endif
+
+template <int NST, int KH, bool STATE_ONLY>
+__global__ void __launch_bounds__(kThreadsTc, 1)
+ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapB,
+            const __grid_constant__ CUtensorMap mapC, const TcParams prm)
+{
+    extern __shared__ uint8_t smem_raw[];
+    // 1024-byte alignment (128-byte swizzle atoms) computed as an offset from the
+    // shared array itself, so every access below stays a shared-memory access
+    const uint32_t smem_pad = ((smem_u32(smem_raw) + 1023u) & ~1023u) - smem_u32(smem_raw);
+    TcSmem<NST> &S = *reinterpret_cast<TcSmem<NST> *>(smem_raw + smem_pad);
+    const int item_idx = blockIdx.x;
+    if (item_idx >= *prm.count) return;
+    const TcItem it = prm.items[item_idx];
+    if (STATE_ONLY && it.seg >= it.nseg - 1) return;   // only non-final segments need end states
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q = warp & 3;                             // SM sub-partition = TMEM lane quarter
+    const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    const int nblk = (it.len + kQ - 1) / kQ;
+    const int nunits = nblk * KH;
+    const int g = it.h0 / prm.heads_per_group;
+    volatile int *abort = &S.abort;
+
+    if (tid == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&S.bc_full[i], 1);
+            mbar_init(&S.bc_empty[i], STATE_ONLY ? 1 : 2);    // state issuer (+ output issuer)
+            mbar_init(&S.x_full[i], 1);
+            mbar_init(&S.x_empty[i], STATE_ONLY ? 2 : 3);     // w o X warps (+ output issuer)
+            mbar_init(&S.xw_full[i], 2);
+            mbar_init(&S.xw_empty[i], 1);
+            mbar_init(&S.pm_full[i], kMaskWarps);
+            mbar_init(&S.pm_empty[i], 1);
+            mbar_init(&S.h_ready[i], 1);
+            mbar_init(&S.hs_full[i], 4);      // per head: H rescaled for its next block
+        }
+        for (int i = 0; i < kCsd; ++i) {
+            mbar_init(&S.cs_full[i], 32);
+            mbar_init(&S.cs_empty[i], STATE_ONLY ? 6 : 6 + kMaskWarps);
+        }
+        mbar_init(&S.cb_full, 1);
+        mbar_init(&S.cb_empty, kMaskWarps);
+        mbar_init(&S.hb_full, 4);
+        mbar_init(&S.hb_empty, 1);
+        mbar_init(&S.y_full, 1);
+        mbar_init(&S.yo_empty, 4);
+        mbar_init(&S.yd_empty, 4);
+        mbar_init(&S.drain_o, 1);
+        mbar_init(&S.drain_s, 1);
+        S.abort = 0;
+        mbar_fence_init();
+    }
+    if (warp == 3) {
+        tmem_alloc(&S.tmem_base, 512);
+        tmem_relinquish();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tb = S.tmem_base;
+#ifdef SSD_TRACE
+    const long long t_start = clock64();
+    long long *const trace_buf = blockIdx.x < kTraceCtas ? g_trace : nullptr;
+#endif
+
+    if (warp == 0) {
+        // ----------------------------------------------------------- cumsum
+        // dt of a unit is loaded before waiting for its ring slot.
+        const int H = prm.H;
+        float Areg[KH];
+#pragma unroll
+        for (int j = 0; j < KH; ++j) Areg[j] = -expf(prm.A_log[it.h0 + j]);
+        bool ok = true;
+        for (int u = 0; u < nunits && ok; ++u) {
+            const int c = u / KH, j = u % KH, slot = u % kCsd;
+            const int row0 = it.tok0 + c * kQ;
+            const int valid = min(kQ, it.len - c * kQ);
+            const int h = it.h0 + j;
+            float r[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int l = lane * 4 + i;
+                r[i] = l < valid ? __bfloat162float(prm.dt[(size_t)(row0 + l) * H + h]) : 0.0f;
+            }
+            float A = Areg[0];
+#pragma unroll
+            for (int jj = 1; jj < KH; ++jj)
+                if (j == jj) A = Areg[jj];
+            if (u >= kCsd) ok = mbar_wait(&S.cs_empty[slot], ((u / kCsd) + 1) & 1, abort);
+            if (!ok) break;
+            // lane owns tokens 4*lane .. 4*lane+3
+            float dl[4], pre[4];
+            float run = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int l = lane * 4 + i;
+                float d = 0.0f;
+                if (l < valid) d = prm.dt_softplus ? fmaxf(r[i], 0.0f) + log1pf(__expf(-fabsf(r[i]))) : r[i];
+                dl[i] = d;
+                run += d * A;
+                pre[i] = run;
+            }
+            float incl = run;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t;
+            }
+            const float excl = incl - run;
+            const float last = __shfl_sync(0xffffffffu, incl, 31);
+            float c2v[4], wv[4], ev[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float csn = excl + pre[i];
+                c2v[i] = csn * kLog2e;
+                wv[i] = ex2_approx((last - csn) * kLog2e) * dl[i];
+                ev[i] = ex2_approx(c2v[i]);
+            }
+            *reinterpret_cast<float4 *>(&S.cs2[slot][lane * 4]) = make_float4(c2v[0], c2v[1], c2v[2], c2v[3]);
+            *reinterpret_cast<float4 *>(&S.dl[slot][lane * 4]) = make_float4(dl[0], dl[1], dl[2], dl[3]);
+            *reinterpret_cast<float4 *>(&S.w[slot][lane * 4]) = make_float4(wv[0], wv[1], wv[2], wv[3]);
+            *reinterpret_cast<float4 *>(&S.e[slot][lane * 4]) = make_float4(ev[0], ev[1], ev[2], ev[3]);
+            if (lane == 0) {
+                S.alpha[slot] = ex2_approx(last * kLog2e);
+                S.ldec[slot] = last;
+            }
+            mbar_arrive(&S.cs_full[slot]);
+            if (lane == 0) SSD_TRACE_EV(6, u);
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------- UMMA issuer: state path
+        // H_j <- H_j + B_c^T (w o X)   (H_j already rescaled by exp(cs_last) by the state warps)
+        if (lane == 0) {
+            const uint32_t id_h = idesc_bf16_f32(128, kP, true, true);
+            const uint32_t lbo_m = NST >= 128 ? 16384u : 0u;   // N = 64: rows 64..127 repeat rows 0..63
+            bool ok = true;
+            for (int c = 0; c < nblk && ok; ++c) {
+                const int bs = c & 1;
+                ok = mbar_wait(&S.bc_full[bs], (c >> 1) & 1, abort);
+                if (!ok) break;
+                const uint32_t sB = smem_u32(S.bc[bs][1][0]);
+                for (int j = 0; j < KH && ok; ++j) {
+                    const int u = c * KH + j, wi = u & 1;
+                    ok = mbar_wait(&S.xw_full[wi], (u >> 1) & 1, abort) && mbar_wait(&S.hs_full[j], c & 1, abort);
+                    SSD_TRACE_EV(15, u);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t sW = smem_u32(S.xw[wi]);
+#pragma unroll
+                    for (int kk = 0; kk < kQ / 16; ++kk)
+                        umma_ss(tb + kColH + 64 * j, sdesc_sw128(sB + kk * 2048, lbo_m, 1024),
+                                sdesc_sw128(sW + kk * 2048, 16384, 1024), id_h, 1);
+                    umma_commit(&S.xw_empty[wi]);
+                    umma_commit(&S.h_ready[j]);
+                    SSD_TRACE_EV(4, u);
+                }
+                umma_commit(&S.bc_empty[bs]);
+            }
+            umma_commit(&S.drain_s);
+            mbar_wait(&S.drain_s, 0, abort, 200000000ull);
+        }
+    } else if (warp == 2) {
+        // ------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&mapX);
+            tma_prefetch_desc(&mapB);
+            if (!STATE_ONLY) tma_prefetch_desc(&mapC);
+            constexpr uint32_t kBoxBytes = 16384;
+            constexpr uint32_t kBcBytes = (STATE_ONLY ? 1 : 2) * (NST / 64) * kBoxBytes;
+            int issued_bc[2] = {-1, -1}, issued_x[2] = {-1, -1};
+            bool ok = true;
+            // L2 prefetch runs kPrefetch blocks ahead of the shared-memory ring
+            auto prefetch = [&](int c) {
+                const int row = it.tok0 + c * kQ;
+                for (int b = 0; b < NST / 64; ++b) {
+                    if (!STATE_ONLY) tma_prefetch_l2_2d(&mapC, g * NST + 64 * b, row);
+                    tma_prefetch_l2_2d(&mapB, g * NST + 64 * b, row);
+                }
+                for (int j = 0; j < KH; ++j) tma_prefetch_l2_2d(&mapX, (it.h0 + j) * kP, row);
+            };
+            for (int c = 0; c < kPrefetch && c < nblk; ++c) prefetch(c);
+            for (int c = 0; c < nblk && ok; ++c) {
+                const int bs = c & 1;
+                if (c + kPrefetch < nblk) prefetch(c + kPrefetch);
+                if (c >= 2) ok = mbar_wait(&S.bc_empty[bs], ((c >> 1) + 1) & 1, abort);
+                if (!ok) break;
+                const int row = it.tok0 + c * kQ;
+                mbar_arrive_expect_tx(&S.bc_full[bs], kBcBytes);
+                for (int b = 0; b < NST / 64; ++b) {
+                    if (!STATE_ONLY) tma_load_2d(S.bc[bs][0][b], &mapC, &S.bc_full[bs], g * NST + 64 * b, row);
+                    tma_load_2d(S.bc[bs][1][b], &mapB, &S.bc_full[bs], g * NST + 64 * b, row);
+                }
+                issued_bc[bs] = c;
+                SSD_TRACE_EV(0, c);
+                for (int j = 0; j < KH; ++j) {
+                    const int u = c * KH + j, xs = u & 1;
+                    if (u >= 2) ok = mbar_wait(&S.x_empty[xs], ((u >> 1) + 1) & 1, abort);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(&S.x_full[xs], kBoxBytes);
+                    tma_load_2d(S.x[xs], &mapX, &S.x_full[xs], (it.h0 + j) * kP, row);
+                    issued_x[xs] = u;
+                    SSD_TRACE_EV(1, u);
+                }
+            }
+            if (!ok) {
+                // drain: wait (bounded) for copies still in flight before the CTA exits
+                for (int i = 0; i < 2; ++i) {
+                    if (issued_bc[i] >= 0) mbar_wait(&S.bc_full[i], (issued_bc[i] >> 1) & 1, abort, 200000000ull);
+                    if (issued_x[i] >= 0) mbar_wait(&S.x_full[i], (issued_x[i] >> 1) & 1, abort, 200000000ull);
+                }
+            }
+        }
+    } else if (warp == 3) {
+        // --------------------------------------------- UMMA issuer: output path
+        if (!STATE_ONLY && lane == 0) {
+            const uint32_t id_cb = idesc_bf16_f32(128, 128, false, false);
+            const uint32_t id_y = idesc_bf16_f32(128, kP, false, true);
+            bool ok = true;
+            // CB = C_c B_c^T into the single CB accumulator
+            auto issue_cb = [&](int c) -> bool {
+                const int bs = c & 1;
+                if (!mbar_wait(&S.bc_full[bs], (c >> 1) & 1, abort)) return false;
+                if (c >= 1 && !mbar_wait(&S.cb_empty, (c - 1) & 1, abort)) return false;
+                tc_fence_after();
+                const uint32_t sC = smem_u32(S.bc[bs][0][0]);
+                const uint32_t sB = smem_u32(S.bc[bs][1][0]);
+#pragma unroll
+                for (int kk = 0; kk < NST / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                    umma_ss(tb + kColCB, sdesc_sw128(sC + off, 16, 1024), sdesc_sw128(sB + off, 16, 1024), id_cb,
+                            kk > 0);
+                }
+                umma_commit(&S.cb_full);
+                SSD_TRACE_EV(2, c);
+                return true;
+            };
+            if (nblk > 0) ok = issue_cb(0);
+            for (int c = 0; c < nblk && ok; ++c) {
+                const int bs = c & 1;
+                const uint32_t sC = smem_u32(S.bc[bs][0][0]);
+                for (int j = 0; j < KH && ok; ++j) {
+                    const int u = c * KH + j, xs = u & 1, pi = u & 1;
+                    // Yo = C Hbf^T
+                    ok = mbar_wait(&S.hb_full, u & 1, abort);
+                    SSD_TRACE_EV(14, u);
+                    ok = ok && (u == 0 || mbar_wait(&S.yo_empty, (u - 1) & 1, abort));
+                    SSD_TRACE_EV(17, u);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t sH = smem_u32(S.hbf);
+#pragma unroll
+                    for (int kk = 0; kk < NST / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                        umma_ss(tb + kColYo, sdesc_sw128(sC + off, 16, 1024),
+                                sdesc_sw128(sH + kk * 2048, 16384, 1024), id_y, kk > 0);
+                    }
+                    umma_commit(&S.hb_empty);
+                    SSD_TRACE_EV(3, u);
+                    // the next block's CB runs while the mask warps finish this block's last head
+                    if (j == KH - 1 && c + 1 < nblk) {
+                        ok = issue_cb(c + 1);
+                        if (!ok) break;
+                    }
+                    // Yd = Pm X
+                    ok = mbar_wait(&S.pm_full[pi], (u >> 1) & 1, abort) &&
+                         mbar_wait(&S.x_full[xs], (u >> 1) & 1, abort) &&
+                         (u == 0 || mbar_wait(&S.yd_empty, (u - 1) & 1, abort));
+                    SSD_TRACE_EV(16, u);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t sX = smem_u32(S.x[xs]);
+#pragma unroll
+                    for (int kk = 0; kk < kQ / 16; ++kk)
+                        umma_ts(tb + kColYd, tb + kColPm + 64 * pi + kk * 8,
+                                sdesc_sw128(sX + kk * 2048, 16384, 1024), id_y, kk > 0);
+                    umma_commit(&S.pm_empty[pi]);
+                    umma_commit(&S.y_full);
+                    umma_commit(&S.x_empty[xs]);
+                    SSD_TRACE_EV(5, u);
+                }
+                umma_commit(&S.bc_empty[bs]);
+            }
+            // every UMMA issued so far has completed before TMEM is released
+            umma_commit(&S.drain_o);
+            mbar_wait(&S.drain_o, 0, abort, 200000000ull);
+        }
+    } else if ((warp >= 4 && warp < 8) || warp == 10 || warp == 11) {
+        // ------------------------------------------------------------- mask
+        // Pm = CB o exp(cs_l - cs_s) delta_s (causal) + D on the diagonal, as
+        // bf16 pairs in TMEM.  Warps 4-7: columns 0..63 for row quarters 0-3;
+        // warps 10-11: columns 64..127 for row quarters 2-3 (quarters 0-1 are
+        // zero there, written once by warps 8-9).
+        if (!STATE_ONLY) {
+            const int half = warp >= 8 ? 1 : 0;
+            const int l = q * 32 + lane;               // row of this thread
+            const int s_begin = half * 64;
+            const int s_hi = min(s_begin + 64, q * 32 + 32);
+            const int npairs = s_hi > s_begin ? (s_hi - s_begin + 31) / 32 : 0;
+            float Dreg[KH];
+#pragma unroll
+            for (int j = 0; j < KH; ++j) Dreg[j] = prm.D ? prm.D[it.h0 + j] : 0.0f;
+            bool ok = true;
+            for (int c = 0; c < nblk && ok; ++c) {
+                ok = mbar_wait(&S.cb_full, c & 1, abort);
+                if (!ok) break;
+                tc_fence_after();
+                for (int j = 0; j < KH; ++j) {
+                    const int u = c * KH + j, slot = u % kCsd, pi = u & 1;
+                    ok = mbar_wait(&S.cs_full[slot], (u / kCsd) & 1, abort) &&
+                         (u < 2 || mbar_wait(&S.pm_empty[pi], ((u >> 1) + 1) & 1, abort));
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (warp == 4 && lane == 0) SSD_TRACE_EV(7, u);
+                    if (warp == 7 && lane == 0) SSD_TRACE_EV(18, u);
+                    const float rowc = S.cs2[slot][l];
+                    float Dh = Dreg[0];
+#pragma unroll
+                    for (int jj = 1; jj < KH; ++jj)
+                        if (j == jj) Dh = Dreg[jj];
+                    const uint32_t pm_col = tb + lane_base + kColPm + 64 * pi + half * 32;
+#pragma unroll
+                    for (int pair = 0; pair < 2; ++pair) {      // 32 columns -> 16 TMEM columns
+                        if (pair < npairs) {                    // warp-uniform
+                            const int s0 = s_begin + pair * 32;
+                            uint32_t packed[16];
+#pragma unroll
+                            for (int sub = 0; sub < 2; ++sub) {
+                                const int s1 = s0 + sub * 16;
+                                uint32_t r[16];
+                                tmem_ld16(tb + lane_base + kColCB + s1, r);
+                                tmem_ld_wait();
+                                if (warp == 7 && lane == 0 && sub == 0) SSD_TRACE_EV(19 + pair, u);
+                                if (j == KH - 1 && pair == npairs - 1 && sub == 1) {
+                                    tc_fence_before();
+                                    __syncwarp();
+                                    if (lane == 0) mbar_arrive(&S.cb_empty);
+                                }
+                                const float4 *cc = reinterpret_cast<const float4 *>(&S.cs2[slot][s1]);
+                                const float4 *dd = reinterpret_cast<const float4 *>(&S.dl[slot][s1]);
+#pragma unroll
+                                for (int i4 = 0; i4 < 4; ++i4) {
+                                    const float4 c4 = cc[i4], d4 = dd[i4];
+                                    const int sa = s1 + 4 * i4;
+                                    // exponents are differences of the block cumsum (<= 0 for s <= l)
+                                    float m0 = __uint_as_float(r[4 * i4 + 0]) * ex2_approx(rowc - c4.x) * d4.x;
+                                    float m1 = __uint_as_float(r[4 * i4 + 1]) * ex2_approx(rowc - c4.y) * d4.y;
+                                    float m2 = __uint_as_float(r[4 * i4 + 2]) * ex2_approx(rowc - c4.z) * d4.z;
+                                    float m3 = __uint_as_float(r[4 * i4 + 3]) * ex2_approx(rowc - c4.w) * d4.w;
+                                    if (sa + 3 >= l) {          // causal edge: s > l is zero, s == l gains D
+                                        m0 = sa + 0 < l ? m0 : (sa + 0 == l ? m0 + Dh : 0.0f);
+                                        m1 = sa + 1 < l ? m1 : (sa + 1 == l ? m1 + Dh : 0.0f);
+                                        m2 = sa + 2 < l ? m2 : (sa + 2 == l ? m2 + Dh : 0.0f);
+                                        m3 = sa + 3 < l ? m3 : (sa + 3 == l ? m3 + Dh : 0.0f);
+                                    }
+                                    packed[8 * sub + 2 * i4] = pack_bf16x2(m0, m1);
+                                    packed[8 * sub + 2 * i4 + 1] = pack_bf16x2(m2, m3);
+                                }
+                            }
+                            tmem_st16(pm_col + pair * 16, packed);
+                        } else {                                // above the diagonal for every row
+                            uint32_t zeros[16];
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) zeros[i] = 0u;
+                            tmem_st16(pm_col + pair * 16, zeros);
+                        }
+                        if (warp == 7 && lane == 0) SSD_TRACE_EV(21 + pair, u);
+                    }
+                    if (j == KH - 1 && npairs == 0) {           // rows with no work still release CB
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&S.cb_empty);
+                    }
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive(&S.pm_full[pi]);
+                        mbar_arrive(&S.cs_empty[slot]);
+                        if (warp == 4) SSD_TRACE_EV(8, u);
+                    }
+                }
+            }
+        }
+    } else if (warp == 8 || warp == 9) {
+        // --------------------------------------------------- w o X (state input)
+        if (!STATE_ONLY) {
+            // the causal mask's columns 64..127 are zero for rows 0..63, in both Pm buffers
+            uint32_t zeros[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) zeros[i] = 0u;
+#pragma unroll
+            for (int pi = 0; pi < 2; ++pi)
+#pragma unroll
+                for (int pair = 0; pair < 2; ++pair) tmem_st16(tb + lane_base + kColPm + 64 * pi + 32 + 16 * pair, zeros);
+            tmem_st_wait();
+            tc_fence_before();
+        }
+        bool ok = true;
+        const int r0 = (warp - 8) * 64 + lane;          // rows r0 and r0 + 32
+        for (int u = 0; u < nunits && ok; ++u) {
+            const int slot = u % kCsd, xs = u & 1, wi = u & 1;
+            ok = mbar_wait(&S.cs_full[slot], (u / kCsd) & 1, abort) &&
+                 mbar_wait(&S.x_full[xs], (u >> 1) & 1, abort) &&
+                 (u < 2 || mbar_wait(&S.xw_empty[wi], ((u >> 1) + 1) & 1, abort));
+            if (!ok) break;
+            if (warp == 8 && lane == 0) SSD_TRACE_EV(25, u);
+            {
+                // all 16 loads in flight before any math or store
+                uint4 v[2][8];
+#pragma unroll
+                for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch)
+                        v[rr][ch] = *reinterpret_cast<const uint4 *>(S.x[xs] + (r0 + 32 * rr) * 128 + ch * 16);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.x_empty[xs]);   // X no longer read by this warp
+#pragma unroll
+                for (int rr = 0; rr < 2; ++rr) {
+                    const int t = r0 + 32 * rr;
+                    const __nv_bfloat162 ws2 = __float2bfloat162_rn(S.w[slot][t]);
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {
+                        __nv_bfloat162 *pv = reinterpret_cast<__nv_bfloat162 *>(&v[rr][ch]);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) pv[i] = __hmul2(pv[i], ws2);
+                        *reinterpret_cast<uint4 *>(S.xw[wi] + t * 128 + ch * 16) = v[rr][ch];   // same swizzled position
+                    }
+                }
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&S.xw_full[wi]);
+                mbar_arrive(&S.cs_empty[slot]);
+                if (warp == 8) SSD_TRACE_EV(11, u);
+            }
+        }
+    } else if (warp >= 12) {
+        // --------------------------------------------------- state + epilogue
+        const int t = q * 32 + lane;                   // TMEM lane: state row n / output row l
+        const int N = NST;
+        const size_t PN = (size_t)kP * N;
+        // initial state of every head: from the caller, from the segment scan, or zero
+        for (int j = 0; j < KH; ++j) {
+            const int h = it.h0 + j;
+            // state-only mode measures each segment from a zero state
+            const float *src = nullptr;
+            if (!STATE_ONLY) {
+                if (it.nseg > 1)
+                    src = prm.segstate + ((size_t)it.gseg * prm.H + h) * PN;
+                else if (prm.init)
+                    src = prm.init + ((size_t)it.seq * prm.H + h) * PN;
+            }
+            const int n = t % N;
+#pragma unroll
+            for (int p0 = 0; p0 < kP; p0 += 16) {
+                uint32_t r[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) r[i] = src ? __float_as_uint(src[(size_t)(p0 + i) * N + n]) : 0u;
+                tmem_st16(tb + lane_base + kColH + 64 * j + p0, r);
+            }
+        }
+        tmem_st_wait();
+        bool ok = true;
+        float ldec_sum[KH];
+#pragma unroll
+        for (int j = 0; j < KH; ++j) ldec_sum[j] = 0.0f;
+
+        // epilogue of unit v: y = Yd + exp(cs_l) Yo for this thread's row
+        auto epilogue = [&](int v) -> bool {
+            const int c = v / KH, j = v % KH, slot = v % kCsd;
+            if (!mbar_wait(&S.y_full, v & 1, abort)) return false;
+            tc_fence_after();
+            if (warp == 12 && lane == 0) SSD_TRACE_EV(12, v);
+            const int valid = min(kQ, it.len - c * kQ);
+            const int tok = it.tok0 + c * kQ + t;
+            const float el = S.e[slot][t];
+            // Yo first (scaled into registers), then Yo goes back to the MMA warp
+            uint32_t yo[64];
+#pragma unroll
+            for (int p0 = 0; p0 < kP; p0 += 16)
+                tmem_ld16(tb + lane_base + kColYo + p0, *reinterpret_cast<uint32_t(*)[16]>(&yo[p0]));
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.yo_empty);
+            if (warp == 12 && lane == 0) SSD_TRACE_EV(26, v);
+            __nv_bfloat16 *dst = prm.y + ((size_t)tok * prm.H + it.h0 + j) * kP;
+#pragma unroll
+            for (int p0 = 0; p0 < kP; p0 += 16) {
+                uint32_t yd[16];
+                tmem_ld16(tb + lane_base + kColYd + p0, yd);
+                tmem_ld_wait();
+                if (p0 == kP - 16) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&S.yd_empty);
+                }
+                if (t < valid) {
+                    uint32_t pk[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        pk[i] = pack_bf16x2(__uint_as_float(yd[2 * i]) + el * __uint_as_float(yo[p0 + 2 * i]),
+                                            __uint_as_float(yd[2 * i + 1]) + el * __uint_as_float(yo[p0 + 2 * i + 1]));
+                    *reinterpret_cast<uint4 *>(dst + p0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    *reinterpret_cast<uint4 *>(dst + p0 + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.cs_empty[slot]);
+            if (warp == 12 && lane == 0) SSD_TRACE_EV(13, v);
+            return true;
+        };
+
+        for (int u = 0; u < nunits && ok; ++u) {
+            const int c = u / KH, j = u % KH, slot = u % kCsd;
+            ok = mbar_wait(&S.cs_full[slot], (u / kCsd) & 1, abort) &&
+                 (c == 0 || mbar_wait(&S.h_ready[j], (c - 1) & 1, abort));
+            if (!ok) break;
+            if (!STATE_ONLY) ok = (u == 0 || mbar_wait(&S.hb_empty, (u - 1) & 1, abort));
+            if (!ok) break;
+            tc_fence_after();
+            if (warp == 12 && lane == 0) SSD_TRACE_EV(9, u);
+            const float alpha = S.alpha[slot];
+            float ld = S.ldec[slot];
+#pragma unroll
+            for (int jj = 0; jj < KH; ++jj)
+                if (j == jj) ldec_sum[jj] += ld;
+            // H pass: Hbf = bf16(H) (rows n, MN-major), H <- alpha * H in place
+            const uint32_t hcol = tb + lane_base + kColH + 64 * j;
+#pragma unroll
+            for (int p0 = 0; p0 < kP; p0 += 16) {
+                uint32_t r[16];
+                tmem_ld16(hcol + p0, r);
+                tmem_ld_wait();
+                if (!STATE_ONLY && t < N) {
+                    uint32_t pk[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+                    *reinterpret_cast<uint4 *>(S.hbf + sw128_offset(t, p0)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    *reinterpret_cast<uint4 *>(S.hbf + sw128_offset(t, p0 + 8)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(alpha * __uint_as_float(r[i]));
+                tmem_st16(hcol + p0, r);
+            }
+            tmem_st_wait();
+            if (!STATE_ONLY) fence_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if (!STATE_ONLY) mbar_arrive(&S.hb_full);
+                mbar_arrive(&S.hs_full[j]);
+                if (STATE_ONLY) mbar_arrive(&S.cs_empty[slot]);
+            }
+            if (warp == 12 && lane == 0) SSD_TRACE_EV(10, u);
+            if (!STATE_ONLY && u >= 1) ok = epilogue(u - 1);
+        }
+        if (!STATE_ONLY && ok && nunits > 0) ok = epilogue(nunits - 1);
+        // end of the segment: the state after the last token
+        if (ok) {
+            for (int j = 0; j < KH; ++j) {
+                ok = mbar_wait(&S.h_ready[j], (nblk - 1) & 1, abort);
+                if (!ok) break;
+                tc_fence_after();
+                const int h = it.h0 + j;
+                float *dst = nullptr;
+                if (STATE_ONLY)
+                    dst = prm.segstate + ((size_t)it.gseg * prm.H + h) * PN;
+                else if (it.seg == it.nseg - 1 && prm.final_states)
+                    dst = prm.final_states + ((size_t)it.seq * prm.H + h) * PN;
+                const uint32_t hcol = tb + lane_base + kColH + 64 * j;
+#pragma unroll
+                for (int p0 = 0; p0 < kP; p0 += 16) {
+                    uint32_t r[16];
+                    tmem_ld16(hcol + p0, r);
+                    tmem_ld_wait();
+                    if (dst && t < N) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) dst[(size_t)(p0 + i) * N + t] = __uint_as_float(r[i]);
+                    }
+                }
+                if (STATE_ONLY && t == 0) prm.seglogdec[(size_t)it.gseg * prm.H + h] = ldec_sum[j];
+            }
+        }
+    }
+
+    // ------------------------------------------------------------ teardown
+    __syncthreads();
+    if (S.abort && tid == 0) record_timeout(prm.status);
+    if (warp == 3) {
+        tc_fence_after();
+        tmem_dealloc(tb, 512);
+    }
+}
+
+// ---------------------------------------------------------------- planning
+// Work items: (sequence, head block, segment).  One block of 1024 threads.
+__global__ void __launch_bounds__(1024)
+tc_plan_kernel(const int32_t *__restrict__ cu_seqlens, int nseq, int seqlen, int seg_len, int n_hb, int KH,
+               TcItem *items, int *count, int max_items, int *status, const float *__restrict__ init,
+               float *__restrict__ final_states, int H, int PN)
+{
+    __shared__ int s_bad, s_carry;
+    __shared__ int s_warp[32];
+    const int tid = threadIdx.x;
+    if (tid == 0) {
+        *status = 0;
+        s_bad = 0;
+        s_carry = 0;
+    }
+    __syncthreads();
+    if (cu_seqlens) {
+        for (int i = tid; i < nseq; i += 1024) {
+            const int a = cu_seqlens[i], b = cu_seqlens[i + 1];
+            if (b < a || (i == 0 && a != 0) || (i == nseq - 1 && b != seqlen)) s_bad = 1;
+        }
+    }
+    __syncthreads();
+    if (s_bad) {
+        if (tid == 0) {
+            set_status(status, kDevBadSeqlens);
+            *count = 0;
+        }
+        return;
+    }
+    for (int base = 0; base < nseq; base += 1024) {
+        const int i = base + tid;
+        int tok0 = 0, len = 0, ns = 0;
+        if (i < nseq) {
+            tok0 = cu_seqlens ? cu_seqlens[i] : i * seqlen;
+            len = cu_seqlens ? cu_seqlens[i + 1] - tok0 : seqlen;
+            ns = (len + seg_len - 1) / seg_len;
+        }
+        int v = ns;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, v, o);
+            if ((tid & 31) >= o) v += t;
+        }
+        if ((tid & 31) == 31) s_warp[tid >> 5] = v;
+        __syncthreads();
+        if (tid < 32) {
+            int w = s_warp[tid];
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, w, o);
+                if (tid >= o) w += t;
+            }
+            s_warp[tid] = w;
+        }
+        __syncthreads();
+        const int incl = v + ((tid >> 5) ? s_warp[(tid >> 5) - 1] : 0) + s_carry;
+        const int gseg0 = incl - ns;
+        if (i < nseq) {
+            for (int sg = 0; sg < ns; ++sg) {
+                const int gs = gseg0 + sg;
+                for (int hb = 0; hb < n_hb; ++hb) {
+                    const int idx = gs * n_hb + hb;
+                    if (idx < max_items) {
+                        TcItem t;
+                        t.seq = i;
+                        t.tok0 = tok0 + sg * seg_len;
+                        t.len = min(seg_len, len - sg * seg_len);
+                        t.gseg = gs;
+                        t.seg = sg;
+                        t.nseg = ns;
+                        t.h0 = hb * KH;
+                        t.pad = 0;
+                        items[idx] = t;
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        if (tid == 1023) s_carry = incl;
+        __syncthreads();
+    }
+    if (tid == 0) *count = min(s_carry * n_hb, max_items);
+    // empty sequences: the final state is the initial state
+    if (final_states) {
+        for (int i = 0; i < nseq; ++i) {
+            const int len = cu_seqlens ? cu_seqlens[i + 1] - cu_seqlens[i] : seqlen;
+            if (len != 0) continue;
+            for (int e = tid; e < H * PN; e += 1024)
+                final_states[(size_t)i * H * PN + e] = init ? init[(size_t)i * H * PN + e] : 0.0f;
+        }
+    }
+}
+
+// Segment scan: entering state of every segment of every sequence,
+// H_in(0) = initial state, H_in(k+1) = exp(ldec_k) H_in(k) + S_k; written in
+// place over the pass-1 end states.
+__global__ void __launch_bounds__(256)
+tc_seg_scan_kernel(const TcItem *__restrict__ items, const int *__restrict__ count, int n_hb, int nseq_items_stride,
+                   float *segstate, const float *__restrict__ seglogdec, const float *__restrict__ init, int H,
+                   int PN)
+{
+    (void)nseq_items_stride;
+    // grid: (first-segment items / n_hb, H, ceil(PN / 256)); blockIdx.x indexes global segments
+    const int gs = blockIdx.x;
+    const int cnt = *count / n_hb;
+    if (gs >= cnt) return;
+    const TcItem it = items[(size_t)gs * n_hb];
+    if (it.seg != 0 || it.nseg < 2) return;   // one thread group per multi-segment sequence
+    const int h = blockIdx.y;
+    const int e = blockIdx.z * 256 + threadIdx.x;
+    if (e >= PN) return;
+    float hv = init ? init[((size_t)it.seq * H + h) * PN + e] : 0.0f;
+    for (int k = 0; k < it.nseg; ++k) {
+        const size_t o = ((size_t)(gs + k) * H + h) * PN + e;
+        const float sv = k < it.nseg - 1 ? segstate[o] : 0.0f;
+        segstate[o] = hv;
+        if (k < it.nseg - 1) hv = fmaf(__expf(seglogdec[(size_t)(gs + k) * H + h]), hv, sv);
+    }
+}
+
+// ------------------------------------------------------------------- host
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 2-D bf16 view [rows][inner] with a {64, 128} box and 128-byte swizzle.
+bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows)
+{
+    auto enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {inner * 2};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct TcPlanShape {
+    int KH, n_hb, seg_len, max_segments, max_items;
+    bool segmented;
+};
+
+int sm_count()
+{
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+TcPlanShape plan_shape(const ssd_fwd_params &p)
+{
+    TcPlanShape s;
+    const int hpg = p.nheads / p.ngroups;
+    s.KH = (hpg % 2 == 0) ? 2 : 1;
+    s.n_hb = p.nheads / s.KH;
+    const int nseq = p.num_seqs > 0 ? p.num_seqs : p.batch;
+    const long long tokens = (long long)p.batch * p.seqlen;
+    const int target = 2 * 148;                       // work items wanted (two per SM)
+    long long seg;
+    if (p.num_seqs > 0) {
+        // packed: bound the longest item so no sequence dominates the makespan
+        seg = (tokens * s.n_hb + target - 1) / target;
+        seg = seg < 1024 ? 1024 : seg;
+    } else {
+        const long long pairs = (long long)p.batch * s.n_hb;
+        long long nseg = pairs >= 148 ? 1 : (target + pairs - 1) / pairs;
+        seg = (p.seqlen + nseg - 1) / (nseg > 0 ? nseg : 1);
+    }
+    seg = (seg + kQ - 1) / kQ * kQ;
+    if (seg < kQ) seg = kQ;
+    s.seg_len = (int)seg;
+    if (p.num_seqs > 0)
+        s.max_segments = (int)((tokens + seg - 1) / seg) + nseq;
+    else
+        s.max_segments = p.batch * (int)((p.seqlen + seg - 1) / seg);
+    s.max_items = s.max_segments * s.n_hb;
+    s.segmented = p.num_seqs > 0 ? (s.seg_len < p.seqlen) : (s.seg_len < p.seqlen);
+    return s;
+}
+
+template <int NST, int KH, bool SO>
+cudaError_t launch_walk(int grid, const CUtensorMap &mX, const CUtensorMap &mB, const CUtensorMap &mC,
+                        const TcParams &prm, cudaStream_t st)
+{
+    const size_t smem = tc_smem_bytes<NST>();
+    cudaError_t e = cudaFuncSetAttribute(ssd_tc_walk<NST, KH, SO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    ssd_tc_walk<NST, KH, SO><<<grid, kThreadsTc, smem, st>>>(mX, mB, mC, prm);
+    return cudaGetLastError();
+}
+
+template <int NST, bool SO>
+cudaError_t launch_walk_kh(int KH, int grid, const CUtensorMap &mX, const CUtensorMap &mB, const CUtensorMap &mC,
+                           const TcParams &prm, cudaStream_t st)
+{
+    return KH == 2 ? launch_walk<NST, 2, SO>(grid, mX, mB, mC, prm, st)
+                   : launch_walk<NST, 1, SO>(grid, mX, mB, mC, prm, st);
+}
+
+template <bool SO>
+cudaError_t launch_walk_any(int N, int KH, int grid, const CUtensorMap &mX, const CUtensorMap &mB,
+                            const CUtensorMap &mC, const TcParams &prm, cudaStream_t st)
+{
+    return N == 128 ? launch_walk_kh<128, SO>(KH, grid, mX, mB, mC, prm, st)
+                    : launch_walk_kh<64, SO>(KH, grid, mX, mB, mC, prm, st);
+}
+
+size_t align256(size_t v) { return (v + 255) / 256 * 256; }
+
+}  // namespace
+
+bool tc_supported(const ssd_fwd_params &p)
+{
+    return p.io_dtype == SSD_DTYPE_BF16 && p.headdim == kP && (p.dstate == 64 || p.dstate == 128) &&
+           p.dt_softplus == 1 && p.chunk_len >= 128 && (long long)p.batch * p.seqlen >= kQ;
+}
+
+size_t tc_workspace_bytes(const ssd_fwd_params &p)
+{
+    const TcPlanShape s = plan_shape(p);
+    size_t b = align256(sizeof(TcItem) * (size_t)s.max_items);
+    if (s.segmented) {
+        b += align256((size_t)s.max_segments * p.nheads * kP * p.dstate * sizeof(float));
+        b += align256((size_t)s.max_segments * p.nheads * sizeof(float));
+    }
+    return b;
+}
+
+int tc_launch_count(const ssd_fwd_params &p) { return plan_shape(p).segmented ? 4 : 2; }
+
+cudaError_t launch_tc(const ssd_fwd_params &p, const Plan &plan, const Dims &d, const TcArgs &a,
+                      cudaStream_t stream, cudaEvent_t prof_begin, cudaEvent_t prof_end)
+{
+    const TcPlanShape s = plan_shape(p);
+    char *ws = static_cast<char *>(a.scratch);
+    TcItem *items = reinterpret_cast<TcItem *>(ws);
+    size_t off = align256(sizeof(TcItem) * (size_t)s.max_items);
+    float *segstate = nullptr, *seglogdec = nullptr;
+    if (s.segmented) {
+        segstate = reinterpret_cast<float *>(ws + off);
+        off += align256((size_t)s.max_segments * p.nheads * kP * p.dstate * sizeof(float));
+        seglogdec = reinterpret_cast<float *>(ws + off);
+    }
+    const long long tokens = (long long)p.batch * p.seqlen;
+    const int PN = kP * p.dstate;
+    const int nseq = plan.nseq;
+    tc_plan_kernel<<<1, 1024, 0, stream>>>(a.cu_seqlens, nseq, p.seqlen, s.seg_len, s.n_hb, s.KH, items,
+                                           plan.count, s.max_items, plan.status, a.init, a.final_states,
+                                           p.nheads, PN);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || tokens == 0) return e;
+
+    CUtensorMap mX, mB, mC;
+    if (!make_map(&mX, a.x, (uint64_t)p.nheads * kP, (uint64_t)tokens) ||
+        !make_map(&mB, a.B, (uint64_t)p.ngroups * p.dstate, (uint64_t)tokens) ||
+        !make_map(&mC, a.C, (uint64_t)p.ngroups * p.dstate, (uint64_t)tokens))
+        return cudaErrorInvalidValue;
+
+    TcParams prm;
+    prm.dt = static_cast<const __nv_bfloat16 *>(a.dt);
+    prm.A_log = a.A_log;
+    prm.D = a.D;
+    prm.init = a.init;
+    prm.y = static_cast<__nv_bfloat16 *>(a.y);
+    prm.final_states = a.final_states;
+    prm.segstate = segstate;
+    prm.seglogdec = seglogdec;
+    prm.items = items;
+    prm.count = plan.count;
+    prm.status = plan.status;
+    prm.H = p.nheads;
+    prm.G = p.ngroups;
+    prm.N = p.dstate;
+    prm.heads_per_group = d.heads_per_group;
+    prm.dt_softplus = p.dt_softplus;
+
+    if (s.segmented) {
+        e = launch_walk_any<true>(p.dstate, s.KH, s.max_items, mX, mB, mC, prm, stream);
+        if (e != cudaSuccess) return e;
+        const dim3 gs(s.max_segments, p.nheads, (PN + 255) / 256);
+        tc_seg_scan_kernel<<<gs, 256, 0, stream>>>(items, plan.count, s.n_hb, 0, segstate, seglogdec, a.init,
+                                                   p.nheads, PN);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (prof_begin) cudaEventRecord(prof_begin, stream);
+    e = launch_walk_any<false>(p.dstate, s.KH, s.max_items, mX, mB, mC, prm, stream);
+    if (prof_end) cudaEventRecord(prof_end, stream);
+    return e;
+}
+
+}  // namespace ssd
+
+#ifdef SSD_TRACE
+extern "C" SSD_API int ssd_trace_enable(long long *buf)
+{
+    return (int)cudaMemcpyToSymbol(ssd::g_trace, &buf, sizeof(buf));
+}
+#endif

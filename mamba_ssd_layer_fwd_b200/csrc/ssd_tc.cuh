@@ -1,0 +1,24 @@
+// Tensor-core (tcgen05 / TMEM / TMA) path of the SSD forward for sm_100a.
+#pragma once
+
+#include "ssd_common.cuh"
+
+namespace ssd {
+
+struct TcArgs {
+    const void *x, *dt, *B, *C;
+    const float *A_log, *D, *init;
+    const int32_t *cu_seqlens;
+    void *y;
+    float *final_states;
+    void *scratch;
+    size_t scratch_bytes;
+};
+
+bool tc_supported(const ssd_fwd_params &p);
+size_t tc_workspace_bytes(const ssd_fwd_params &p);
+int tc_launch_count(const ssd_fwd_params &p);
+cudaError_t launch_tc(const ssd_fwd_params &p, const Plan &plan, const Dims &d, const TcArgs &a,
+                      cudaStream_t stream, cudaEvent_t prof_begin, cudaEvent_t prof_end);
+
+}  // namespace ssd

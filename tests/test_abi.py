@@ -1,0 +1,99 @@
+"""The C-ABI library: it loads, exports every declared entry point, and its
+host-side validation rejects bad arguments before touching the device (no GPU
+needed: every call here fails validation or only queries sizes)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import mamba_ssd_layer_fwd_b200 as ssd
+from mamba_ssd_layer_fwd_b200 import build as ssd_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    ssd_build.build()
+    return ssd.library()
+
+
+def declared_symbols():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            body = src.split("#endif\n", 1)[-1] if "#define SSD_API" in src else src
+            names += re.findall(r"^SSD_API\s+[\w\s\*]*?\b(\w+)\s*\(", body, flags=re.M)
+    return sorted(set(names))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_symbols()
+    assert "ssd_fwd" in names and "ssd_fwd_workspace_size" in names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+    assert lib.ssd_abi_version() == 1
+
+
+def test_only_abi_symbols_exported(lib):
+    # the .so hides everything but the C ABI (-fvisibility=hidden)
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", ssd.library_path()], capture_output=True,
+                         text=True).stdout
+    ours = {l.split()[-1] for l in out.splitlines() if " T " in l and l.split()[-1].startswith("ssd_")}
+    assert ours == set(declared_symbols())
+
+
+def params(**kw):
+    base = dict(batch=2, seqlen=2048, nheads=24, headdim=64, dstate=64, ngroups=1, chunk_len=256,
+                num_seqs=0, io_dtype="bf16", dt_softplus=True, path="auto")
+    base.update(kw)
+    return ssd.make_params(**base)
+
+
+def test_workspace_size_valid_and_invalid(lib):
+    assert ssd.workspace_size(params()) > 0
+    assert ssd.workspace_size(params(path="simt")) > 0
+    for bad in (dict(nheads=24, ngroups=5), dict(chunk_len=100), dict(batch=0), dict(headdim=0),
+                dict(num_seqs=3, batch=2), dict(dstate=300), dict(headdim=256)):
+        assert ssd.workspace_size(params(**bad)) == 0, bad
+
+
+def test_resolved_path_and_launch_count(lib):
+    p = params(path="simt")
+    assert ssd.resolved_path(p) == "simt"
+    assert ssd.launch_count(p) == 5
+    assert ssd.resolved_path(params(io_dtype="f32")) == "simt"
+
+
+def _call(lib, p, **ptrs):
+    args = dict(x=16, dt=16, A_log=16, B=16, C=16, D=None, init=None, cu=None, y=16, final=None,
+                ws=256, ws_bytes=1 << 40)
+    args.update(ptrs)
+    return lib.ssd_fwd(ctypes.byref(p), args["x"], args["dt"], args["A_log"], args["B"], args["C"],
+                       args["D"], args["init"], args["cu"], args["y"], args["final"], args["ws"],
+                       args["ws_bytes"], None)
+
+
+def test_validation_errors(lib):
+    INVALID, UNSUPPORTED = -1, -2
+    assert lib.ssd_fwd(None, 16, 16, 16, 16, 16, None, None, None, 16, None, 256, 1 << 40, None) == INVALID
+    assert _call(lib, params(), x=None) == INVALID
+    assert _call(lib, params(), y=None) == INVALID
+    assert _call(lib, params(), ws=None) == INVALID
+    assert _call(lib, params(), x=24) == INVALID                 # misaligned
+    assert _call(lib, params(), ws=128) == INVALID               # workspace not 256-aligned
+    assert _call(lib, params(), ws_bytes=16) == INVALID          # workspace too small
+    assert _call(lib, params(nheads=6, ngroups=4)) == INVALID
+    assert _call(lib, params(chunk_len=32)) == INVALID
+    assert _call(lib, params(num_seqs=2, batch=1)) == INVALID    # cu_seqlens missing
+    assert _call(lib, params(), cu=16) == INVALID                # cu_seqlens without num_seqs
+    assert _call(lib, params(headdim=200)) == UNSUPPORTED
+    assert _call(lib, params(path="tensor", io_dtype="f32")) == UNSUPPORTED
+
+
+def test_status_strings(lib):
+    for code in ssd.STATUS:
+        assert lib.ssd_status_string(code)

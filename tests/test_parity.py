@@ -1,0 +1,157 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 CPU oracle,
+element by element, on seeded inputs. Tolerance: max|dy| / max|y_oracle| <=
+2e-2 for bf16 inputs, <= 1e-4 for float32; final states to the same bound."""
+import numpy as np
+import pytest
+
+import oracle
+import ssd_inputs
+from _helpers import BF16_TOL, F32_TOL, rel_max_err, run_gpu, small_inputs
+
+pytestmark = pytest.mark.gpu
+
+PATHS = ["simt", "tensor"]
+
+
+def _maybe_skip_path(inp, path):
+    import mamba_ssd_layer_fwd_b200 as ssd
+    x, B = inp["x"], inp["B"]
+    nseq = 0 if inp.get("cu_seqlens") is None else len(inp["cu_seqlens"]) - 1
+    p = ssd.make_params(batch=x.shape[0], seqlen=x.shape[1], nheads=x.shape[2], headdim=x.shape[3],
+                        dstate=B.shape[3], ngroups=B.shape[2], chunk_len=inp["chunk_len"],
+                        num_seqs=nseq, io_dtype=inp["io_dtype"], path=path)
+    if ssd.resolved_path(p) != path:
+        pytest.skip(f"{path} path does not take this shape")
+
+
+def check_full(inp, path="auto", chunk_len=None, tol=None):
+    tol = tol or (F32_TOL if inp["io_dtype"] == "f32" else BF16_TOL)
+    y, fin = run_gpu(inp, path=path, chunk_len=chunk_len)
+    y_ref, fin_ref = oracle.recurrence(inp)
+    ey, ef = rel_max_err(y, y_ref), rel_max_err(fin, fin_ref)
+    assert ey <= tol, f"y rel err {ey:.3e} > {tol}"
+    assert ef <= tol, f"final-state rel err {ef:.3e} > {tol}"
+    return y, fin, ey, ef
+
+
+# ------------------------------------------------------------- tiny float32
+
+def test_tiny_f32_workload():
+    """The tiny float32 workload (T=256, H=2, P=N=16, chunk 64) to 1e-4."""
+    inp = ssd_inputs.make_inputs(ssd_inputs.workload("tiny_f32", with_final_states=True))
+    check_full(inp)
+
+
+@pytest.mark.parametrize("Q", [64, 128, 256])
+def test_f32_ragged_with_initial_state(Q):
+    inp = small_inputs(batch=2, seqlen=333, H=3, P=16, N=24, G=1, Q=Q, io="f32", init=True,
+                       xbc_std=1.0, dt_shift=2.0, a_log_hi=1.5)
+    check_full(inp)
+
+
+# ----------------------------------------------------------------- bf16
+
+@pytest.mark.parametrize("path", PATHS)
+@pytest.mark.parametrize("N,G,H", [(64, 1, 4), (128, 1, 6), (256, 2, 4), (128, 4, 8)])
+def test_bf16_shapes_ragged(path, N, G, H):
+    inp = small_inputs(batch=2, seqlen=700, H=H, P=64, N=N, G=G, Q=256, init=True, seed=N + G)
+    _maybe_skip_path(inp, path)
+    check_full(inp, path=path)
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_bf16_varlen_with_states(path):
+    lens = [1, 255, 256, 257, 0, 700, 64, 3]
+    inp = small_inputs(H=4, P=64, N=128, G=1, Q=256, varlen=lens, init=True, seed=3)
+    _maybe_skip_path(inp, path)
+    check_full(inp, path=path)
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_chunk_length_invariance(path):
+    """Sec. 6: the block decomposition is exact for any chunk length."""
+    inp = small_inputs(batch=1, seqlen=1024, H=4, P=64, N=64, G=1, Q=256, init=True, seed=5)
+    outs = []
+    for Q in (64, 128, 256):
+        inp["chunk_len"] = Q
+        try:
+            _maybe_skip_path(inp, path)
+        except pytest.skip.Exception:
+            continue
+        y, fin, _, _ = check_full(inp, path=path, chunk_len=Q)
+        outs.append(y)
+    for y in outs[1:]:
+        assert rel_max_err(y, outs[0]) <= 2 * BF16_TOL
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_decay_one_and_zero(path):
+    inp = small_inputs(batch=1, seqlen=520, H=2, P=64, N=64, G=1, Q=256, init=True, seed=6)
+    _maybe_skip_path(inp, path)
+    inp["A_log"] = np.array([-np.inf, 30.0], dtype=np.float32)   # head 0: a == 1, head 1: a == 0
+    check_full(inp, path=path)
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_single_token_and_empty(path):
+    inp = small_inputs(batch=3, seqlen=1, H=2, P=64, N=64, G=1, Q=256, init=True, seed=7)
+    _maybe_skip_path(inp, path)
+    check_full(inp, path=path)
+
+
+def test_zero_length_batch_passes_initial_state():
+    inp = small_inputs(batch=2, seqlen=0, H=2, P=64, N=64, G=1, Q=256, init=True, seed=8)
+    y, fin = run_gpu(inp)
+    assert y.size == 0
+    np.testing.assert_array_equal(fin, inp["initial_states"].astype(np.float64))
+
+
+def test_deterministic():
+    inp = small_inputs(batch=1, seqlen=900, H=4, P=64, N=128, G=1, Q=256, init=True, seed=9)
+    a, fa = run_gpu(inp)
+    b, fb = run_gpu(inp)
+    assert np.array_equal(a, b) and np.array_equal(fa, fb)
+
+
+def test_bad_cu_seqlens_reported_in_status():
+    import torch
+    import mamba_ssd_layer_fwd_b200 as ssd
+    from _helpers import to_device
+    inp = small_inputs(H=2, P=64, N=64, G=1, Q=256, varlen=[100, 100], init=False, seed=10)
+    t = to_device(inp)
+    t["cu_seqlens"] = torch.tensor([0, 150, 120], dtype=torch.int32, device="cuda")
+    with pytest.raises(ssd.SsdError) as e:
+        ssd.ssd_fwd(t["x"], t["dt"], t["A_log"], t["B"], t["C"], t["D"], chunk_len=256,
+                    cu_seqlens=t["cu_seqlens"], check_status=True)
+    assert e.value.code == -5
+
+
+# ------------------------------------------------ benchmark shapes, sampled
+
+SAMPLED = {
+    "small_bf16": [(0, 0), (1, 23), (0, 11)],
+    "mamba2_2p7b": [(0, 0), (7, 79), (3, 40), (5, 13)],
+    "long16k_gva": [(0, 0), (0, 31), (0, 17)],
+    "varlen32k": [(0, 0), (15, 47), (7, 20), (11, 3)],
+}
+
+
+@pytest.mark.parametrize("name", list(SAMPLED))
+def test_benchmark_workload_sampled(name):
+    """Full-size benchmark shapes in the bench's launch configuration; the
+    oracle recomputes sampled (sequence, head) pairs."""
+    w = ssd_inputs.workload(name, with_final_states=True)
+    inp = ssd_inputs.make_inputs(w)
+    y, fin = run_gpu(inp)
+    pairs = SAMPLED[name]
+    ys, fs = oracle.recurrence_pairs(inp, pairs)
+    bounds = ssd_inputs.seq_bounds(inp)
+    H, P = inp["x"].shape[2], inp["x"].shape[3]
+    yf = y.reshape(-1, H, P)
+    for (s, h), yr, fr in zip(pairs, ys, fs):
+        t0, n = bounds[s]
+        ey = rel_max_err(yf[t0:t0 + n, h], yr)
+        ef = rel_max_err(fin[s, h], fr)
+        assert ey <= BF16_TOL, f"{name} pair {(s, h)}: y rel err {ey:.3e}"
+        assert ef <= BF16_TOL, f"{name} pair {(s, h)}: final rel err {ef:.3e}"
+    assert np.all(np.isfinite(y))
