@@ -114,6 +114,34 @@ SSD_API ssd_status ssd_fwd(const ssd_fwd_params *p,
                    void *y, float *final_states,
                    void *workspace, size_t workspace_bytes, void *stream);
 
+/* Size of the fixed scratch array behind ssd_fwd_noalloc: 16 MiB of device
+ * memory on every GPU that loads this library, held until the process exits. */
+#define SSD_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* Allocation-free SSD forward, for callers that cannot allocate device memory
+ * (inside an allocator's own callbacks, in a real-time loop that must not take
+ * allocator locks or risk running out of memory mid-run, in a runtime that
+ * only lends out the tensors it owns).  No counterpart in the paper: it is the
+ * same operation as ssd_fwd, with the workspace taken from a file-scope
+ * __device__ array of SSD_NOALLOC_SCRATCH_BYTES instead of the caller.
+ *   - Arguments are those of ssd_fwd minus the workspace; inputs and outputs
+ *     are still the caller's device buffers.
+ *   - Returns SSD_ERR_UNSUPPORTED (nothing launched) when the problem needs
+ *     more workspace than SSD_NOALLOC_SCRATCH_BYTES (ssd_fwd_workspace_size).
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *   - The first call on a device looks up the array's address with that
+ *     device current; make it before any stream capture.
+ *   - Every call shares the array.  The kernels clear what must start at zero
+ *     and overwrite the rest before reading it, but calls that overlap on the
+ *     GPU (other streams, other threads on the same device) race on it.
+ *   - sync_status != 0: synchronise `stream` and return the device-side status
+ *     (what ssd_get_status reports for ssd_fwd). */
+SSD_API ssd_status ssd_fwd_noalloc(const ssd_fwd_params *p,
+                   const void *x, const void *dt, const float *A_log,
+                   const void *B, const void *C, const float *D,
+                   const float *initial_states, const int32_t *cu_seqlens,
+                   void *y, float *final_states, void *stream, int sync_status);
+
 /* Device-side status of the last ssd_fwd that used `workspace` on `stream`:
  * synchronises `stream`, then returns SSD_OK, SSD_ERR_TIMEOUT or
  * SSD_ERR_BAD_SEQLENS (or SSD_ERR_CUDA if the copy fails). */
