@@ -86,9 +86,11 @@ struct TcParams {
 template <int NST>
 struct __align__(1024) TcSmem {
     static constexpr int kBoxes = NST / 64;
-    uint8_t bc[2][2][kBoxes][16384];   // [stage][0 = C, 1 = B][64-column box][128 rows x 128 B]
+    static constexpr int kStages = NST >= 256 ? 1 : 2;   // B/C ring depth (dstate 256: one stage fits)
+    static constexpr int kXw = NST >= 256 ? 1 : 2;       // w o X ring depth
+    uint8_t bc[kStages][2][kBoxes][16384];   // [stage][0 = C, 1 = B][64-column box][128 rows x 128 B]
     uint8_t x[2][16384];               // X blocks (ring over (block, head))
-    uint8_t xw[2][16384];              // w o X (ring over (block, head))
+    uint8_t xw[kXw][16384];            // w o X (ring over (block, head))
     uint8_t hbf[NST * 128];            // bf16(H)^T: rows n, 64 p per 128 B row
     float cs2[kCsd][kQ];               // log2-scaled inclusive cumsum of delta*A
     float dl[kCsd][kQ];                // delta_s (0 on padding rows)
@@ -151,6 +153,8 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
     const int nunits = nblk * KH;
     const int g = it.h0 / prm.heads_per_group;
     volatile int *abort = &S.abort;
+    constexpr int kSt = TcSmem<NST>::kStages, kXwD = TcSmem<NST>::kXw;
+    constexpr int kMT = NST >= 256 ? 2 : 1;        // 128-row state tiles per head (H^T rows = n)
 
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
@@ -265,21 +269,24 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             const uint32_t lbo_m = NST >= 128 ? 16384u : 0u;   // N = 64: rows 64..127 repeat rows 0..63
             bool ok = true;
             for (int c = 0; c < nblk && ok; ++c) {
-                const int bs = c & 1;
-                ok = mbar_wait(&S.bc_full[bs], (c >> 1) & 1, abort);
+                const int bs = c % kSt;
+                ok = mbar_wait(&S.bc_full[bs], (c / kSt) & 1, abort);
                 if (!ok) break;
                 const uint32_t sB = smem_u32(S.bc[bs][1][0]);
                 for (int j = 0; j < KH && ok; ++j) {
-                    const int u = c * KH + j, wi = u & 1;
-                    ok = mbar_wait(&S.xw_full[wi], (u >> 1) & 1, abort) && mbar_wait(&S.hs_full[j], c & 1, abort);
+                    const int u = c * KH + j, wi = u % kXwD;
+                    ok = mbar_wait(&S.xw_full[wi], (u / kXwD) & 1, abort) && mbar_wait(&S.hs_full[j], c & 1, abort);
                     SSD_TRACE_EV(15, u);
                     if (!ok) break;
                     tc_fence_after();
                     const uint32_t sW = smem_u32(S.xw[wi]);
 #pragma unroll
-                    for (int kk = 0; kk < kQ / 16; ++kk)
-                        umma_ss(tb + kColH + 64 * j, sdesc_sw128(sB + kk * 2048, lbo_m, 1024),
-                                sdesc_sw128(sW + kk * 2048, 16384, 1024), id_h, 1);
+                    for (int mt = 0; mt < kMT; ++mt)
+#pragma unroll
+                        for (int kk = 0; kk < kQ / 16; ++kk)
+                            umma_ss(tb + kColH + 64 * (j * kMT + mt),
+                                    sdesc_sw128(sB + mt * 32768 + kk * 2048, lbo_m, 1024),
+                                    sdesc_sw128(sW + kk * 2048, 16384, 1024), id_h, 1);
                     umma_commit(&S.xw_empty[wi]);
                     umma_commit(&S.h_ready[j]);
                     SSD_TRACE_EV(4, u);
@@ -310,9 +317,9 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             };
             for (int c = 0; c < kPrefetch && c < nblk; ++c) prefetch(c);
             for (int c = 0; c < nblk && ok; ++c) {
-                const int bs = c & 1;
+                const int bs = c % kSt;
                 if (c + kPrefetch < nblk) prefetch(c + kPrefetch);
-                if (c >= 2) ok = mbar_wait(&S.bc_empty[bs], ((c >> 1) + 1) & 1, abort);
+                if (c >= kSt) ok = mbar_wait(&S.bc_empty[bs], ((c / kSt) + 1) & 1, abort);
                 if (!ok) break;
                 const int row = it.tok0 + c * kQ;
                 mbar_arrive_expect_tx(&S.bc_full[bs], kBcBytes);
@@ -335,7 +342,8 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             if (!ok) {
                 // drain: wait (bounded) for copies still in flight before the CTA exits
                 for (int i = 0; i < 2; ++i) {
-                    if (issued_bc[i] >= 0) mbar_wait(&S.bc_full[i], (issued_bc[i] >> 1) & 1, abort, 200000000ull);
+                    if (i < kSt && issued_bc[i] >= 0)
+                        mbar_wait(&S.bc_full[i], (issued_bc[i] / kSt) & 1, abort, 200000000ull);
                     if (issued_x[i] >= 0) mbar_wait(&S.x_full[i], (issued_x[i] >> 1) & 1, abort, 200000000ull);
                 }
             }
@@ -348,8 +356,8 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             bool ok = true;
             // CB = C_c B_c^T into the single CB accumulator
             auto issue_cb = [&](int c) -> bool {
-                const int bs = c & 1;
-                if (!mbar_wait(&S.bc_full[bs], (c >> 1) & 1, abort)) return false;
+                const int bs = c % kSt;
+                if (!mbar_wait(&S.bc_full[bs], (c / kSt) & 1, abort)) return false;
                 if (c >= 1 && !mbar_wait(&S.cb_empty, (c - 1) & 1, abort)) return false;
                 tc_fence_after();
                 const uint32_t sC = smem_u32(S.bc[bs][0][0]);
@@ -364,10 +372,16 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                 SSD_TRACE_EV(2, c);
                 return true;
             };
-            if (nblk > 0) ok = issue_cb(0);
+            // With two B/C stages the next block's CB is issued early (below); with one
+            // stage its operands only arrive after this block is released, so it waits.
+            if (kSt > 1 && nblk > 0) ok = issue_cb(0);
             for (int c = 0; c < nblk && ok; ++c) {
-                const int bs = c & 1;
+                const int bs = c % kSt;
                 const uint32_t sC = smem_u32(S.bc[bs][0][0]);
+                if (kSt == 1) {
+                    ok = issue_cb(c);
+                    if (!ok) break;
+                }
                 for (int j = 0; j < KH && ok; ++j) {
                     const int u = c * KH + j, xs = u & 1, pi = u & 1;
                     // Yo = C Hbf^T
@@ -387,7 +401,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                     umma_commit(&S.hb_empty);
                     SSD_TRACE_EV(3, u);
                     // the next block's CB runs while the mask warps finish this block's last head
-                    if (j == KH - 1 && c + 1 < nblk) {
+                    if (kSt > 1 && j == KH - 1 && c + 1 < nblk) {
                         ok = issue_cb(c + 1);
                         if (!ok) break;
                     }
@@ -528,10 +542,10 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
         bool ok = true;
         const int r0 = (warp - 8) * 64 + lane;          // rows r0 and r0 + 32
         for (int u = 0; u < nunits && ok; ++u) {
-            const int slot = u % kCsd, xs = u & 1, wi = u & 1;
+            const int slot = u % kCsd, xs = u & 1, wi = u % kXwD;
             ok = mbar_wait(&S.cs_full[slot], (u / kCsd) & 1, abort) &&
                  mbar_wait(&S.x_full[xs], (u >> 1) & 1, abort) &&
-                 (u < 2 || mbar_wait(&S.xw_empty[wi], ((u >> 1) + 1) & 1, abort));
+                 (u < kXwD || mbar_wait(&S.xw_empty[wi], ((u / kXwD) + 1) & 1, abort));
             if (!ok) break;
             if (warp == 8 && lane == 0) SSD_TRACE_EV(25, u);
             {
@@ -581,13 +595,16 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                 else if (prm.init)
                     src = prm.init + ((size_t)it.seq * prm.H + h) * PN;
             }
-            const int n = t % N;
 #pragma unroll
-            for (int p0 = 0; p0 < kP; p0 += 16) {
-                uint32_t r[16];
+            for (int mt = 0; mt < kMT; ++mt) {
+                const int n = kMT > 1 ? t + 128 * mt : t % N;   // N = 64: lanes 64..127 mirror 0..63
 #pragma unroll
-                for (int i = 0; i < 16; ++i) r[i] = src ? __float_as_uint(src[(size_t)(p0 + i) * N + n]) : 0u;
-                tmem_st16(tb + lane_base + kColH + 64 * j + p0, r);
+                for (int p0 = 0; p0 < kP; p0 += 16) {
+                    uint32_t r[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) r[i] = src ? __float_as_uint(src[(size_t)(p0 + i) * N + n]) : 0u;
+                    tmem_st16(tb + lane_base + kColH + 64 * (j * kMT + mt) + p0, r);
+                }
             }
         }
         tmem_st_wait();
@@ -657,23 +674,28 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             for (int jj = 0; jj < KH; ++jj)
                 if (j == jj) ldec_sum[jj] += ld;
             // H pass: Hbf = bf16(H) (rows n, MN-major), H <- alpha * H in place
-            const uint32_t hcol = tb + lane_base + kColH + 64 * j;
 #pragma unroll
-            for (int p0 = 0; p0 < kP; p0 += 16) {
-                uint32_t r[16];
-                tmem_ld16(hcol + p0, r);
-                tmem_ld_wait();
-                if (!STATE_ONLY && t < N) {
-                    uint32_t pk[8];
+            for (int mt = 0; mt < kMT; ++mt) {
+                const uint32_t hcol = tb + lane_base + kColH + 64 * (j * kMT + mt);
+                const int n = t + 128 * mt;
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-                    *reinterpret_cast<uint4 *>(S.hbf + sw128_offset(t, p0)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    *reinterpret_cast<uint4 *>(S.hbf + sw128_offset(t, p0 + 8)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                for (int p0 = 0; p0 < kP; p0 += 16) {
+                    uint32_t r[16];
+                    tmem_ld16(hcol + p0, r);
+                    tmem_ld_wait();
+                    if (!STATE_ONLY && n < N) {
+                        uint32_t pk[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+                        *reinterpret_cast<uint4 *>(S.hbf + sw128_offset(n, p0)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        *reinterpret_cast<uint4 *>(S.hbf + sw128_offset(n, p0 + 8)) =
+                            make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                    }
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(alpha * __uint_as_float(r[i]));
+                    tmem_st16(hcol + p0, r);
                 }
-#pragma unroll
-                for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(alpha * __uint_as_float(r[i]));
-                tmem_st16(hcol + p0, r);
             }
             tmem_st_wait();
             if (!STATE_ONLY) fence_async_smem();
@@ -700,15 +722,19 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                     dst = prm.segstate + ((size_t)it.gseg * prm.H + h) * PN;
                 else if (it.seg == it.nseg - 1 && prm.final_states)
                     dst = prm.final_states + ((size_t)it.seq * prm.H + h) * PN;
-                const uint32_t hcol = tb + lane_base + kColH + 64 * j;
 #pragma unroll
-                for (int p0 = 0; p0 < kP; p0 += 16) {
-                    uint32_t r[16];
-                    tmem_ld16(hcol + p0, r);
-                    tmem_ld_wait();
-                    if (dst && t < N) {
+                for (int mt = 0; mt < kMT; ++mt) {
+                    const uint32_t hcol = tb + lane_base + kColH + 64 * (j * kMT + mt);
+                    const int n = t + 128 * mt;
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) dst[(size_t)(p0 + i) * N + t] = __uint_as_float(r[i]);
+                    for (int p0 = 0; p0 < kP; p0 += 16) {
+                        uint32_t r[16];
+                        tmem_ld16(hcol + p0, r);
+                        tmem_ld_wait();
+                        if (dst && n < N) {
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) dst[(size_t)(p0 + i) * N + n] = __uint_as_float(r[i]);
+                        }
                     }
                 }
                 if (STATE_ONLY && t == 0) prm.seglogdec[(size_t)it.gseg * prm.H + h] = ldec_sum[j];
@@ -893,7 +919,8 @@ TcPlanShape plan_shape(const ssd_fwd_params &p)
 {
     TcPlanShape s;
     const int hpg = p.nheads / p.ngroups;
-    s.KH = (hpg % 2 == 0) ? 2 : 1;
+    // two heads per CTA share B/C tiles; dstate 256 leaves TMEM for one head's state
+    s.KH = (hpg % 2 == 0 && p.dstate <= 128) ? 2 : 1;
     s.n_hb = p.nheads / s.KH;
     const int nseq = p.num_seqs > 0 ? p.num_seqs : p.batch;
     const long long tokens = (long long)p.batch * p.seqlen;
@@ -944,6 +971,7 @@ template <bool SO>
 cudaError_t launch_walk_any(int N, int KH, int grid, const CUtensorMap &mX, const CUtensorMap &mB,
                             const CUtensorMap &mC, const TcParams &prm, cudaStream_t st)
 {
+    if (N == 256) return launch_walk<256, 1, SO>(grid, mX, mB, mC, prm, st);
     return N == 128 ? launch_walk_kh<128, SO>(KH, grid, mX, mB, mC, prm, st)
                     : launch_walk_kh<64, SO>(KH, grid, mX, mB, mC, prm, st);
 }
@@ -954,7 +982,8 @@ size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
 bool tc_supported(const ssd_fwd_params &p)
 {
-    return p.io_dtype == SSD_DTYPE_BF16 && p.headdim == kP && (p.dstate == 64 || p.dstate == 128) &&
+    return p.io_dtype == SSD_DTYPE_BF16 && p.headdim == kP &&
+           (p.dstate == 64 || p.dstate == 128 || p.dstate == 256) &&
            p.dt_softplus == 1 && p.chunk_len >= 128 && (long long)p.batch * p.seqlen >= kQ;
 }
 

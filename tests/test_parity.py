@@ -60,6 +60,14 @@ def test_bf16_shapes_ragged(path, N, G, H):
 
 
 @pytest.mark.parametrize("path", PATHS)
+def test_bf16_dstate256_long_segments(path):
+    """dstate 256 with several 128-token blocks per segment (one B/C stage)."""
+    inp = small_inputs(batch=1, seqlen=3000, H=2, P=64, N=256, G=1, Q=256, init=True, seed=31)
+    _maybe_skip_path(inp, path)
+    check_full(inp, path=path)
+
+
+@pytest.mark.parametrize("path", PATHS)
 def test_bf16_varlen_with_states(path):
     lens = [1, 255, 256, 257, 0, 700, 64, 3]
     inp = small_inputs(H=4, P=64, N=128, G=1, Q=256, varlen=lens, init=True, seed=3)
