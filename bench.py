@@ -32,6 +32,7 @@ sys.path.insert(0, ROOT)
 import ssd_inputs  # noqa: E402
 
 L2_FLUSH_BYTES = 512 << 20        # > 4x the 126 MB L2
+METRIC = "SSD fwd tokens/s at 1 B200; % of BF16 tensor-core / HBM roofline"
 FALLBACK_HBM_GBS = 6650.0
 THROTTLE_BITS = {
     0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
@@ -187,6 +188,25 @@ def cpu_oracle_rate(inp: dict, budget_s: float = 10.0):
 
 # ------------------------------------------------------------------ helpers
 
+def max_over_ranks(values, device=None):
+    """Element-wise max of a list of floats over all ranks of the default
+    process group (identity without one). Every rank calls it at the same
+    point, in warm-up, timing and error paths alike."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def whole_job_throughput(tokens_per_rank: int, world: int, step_ms_max: float) -> float:
+    """Weak scaling: every rank runs its own copy of the workload; the job's
+    throughput is all ranks' tokens over the slowest rank's step time."""
+    return tokens_per_rank * world / (step_ms_max * 1e-3)
+
+
 def make_workload(args):
     w = ssd_inputs.workload(args.workload)
     return ssd_inputs.make_inputs(w, seed=args.seed)
@@ -218,7 +238,7 @@ def run_reference(args):
             per_step.append(rate)
     value = float(statistics.median(per_step))
     line = {
-        "impl": "reference", "metric": "SSD fwd tokens/s", "value": value, "unit": "tokens/s",
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000.0 * tokens / value, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
@@ -305,12 +325,7 @@ def run_ours(args):
     clocks = sampler.stop() if rank == 0 else None
     step_ms = [ev[i][0].elapsed_time(ev[i][3]) for i in range(K)]
     main_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
-    ms = statistics.mean(step_ms)
-    kms = statistics.mean(main_ms)
-    if world > 1:
-        t = torch.tensor([ms, kms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, kms = float(t[0]), float(t[1])
+    ms, kms = max_over_ranks([statistics.mean(step_ms), statistics.mean(main_ms)], dev)
 
     # end to end: pinned host inputs -> device -> ssd_fwd -> result back to pinned host memory
     y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
@@ -333,15 +348,11 @@ def run_ours(args):
         torch.cuda.synchronize()
         if i >= args.warmup:
             e2e_ms.append(e0.elapsed_time(e1))
-    e2e = statistics.mean(e2e_ms)
-    if world > 1:
-        t = torch.tensor([e2e], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e = float(t[0])
+    e2e = max_over_ranks([statistics.mean(e2e_ms)], dev)[0]
 
     tokens = inp["x"].shape[0] * inp["x"].shape[1]
     total_tokens = tokens * world
-    value = total_tokens / (ms * 1e-3)
+    value = whole_job_throughput(tokens, world, ms)
     alg_bytes = algorithmic_bytes(inp)
     flops = algorithmic_flops(inp)
     peak, peak_kind = measured_peaks()
@@ -354,7 +365,7 @@ def run_ours(args):
             rate, cores, desc, _ = cpu_oracle_rate(inp, budget_s=args.ref_seconds)
             cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc}
         line = {
-            "metric": "SSD fwd tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": inp["io_dtype"],
             "data": "synthetic (seeded generator, value distributions of the workload)",
@@ -365,7 +376,7 @@ def run_ours(args):
                          "peak_source": f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"},
             "tflops": flops / (ms * 1e-3) / 1e12,
             "cpu_baseline": cpu,
-            "e2e": {"value": total_tokens / (e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "e2e": {"value": whole_job_throughput(tokens, world, e2e), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": launches_per_step * K,
             "clocks": clocks,

@@ -96,6 +96,9 @@ typedef struct ssd_fwd_params {
     ssd_path path;
     void *prof_begin;           /* optional cudaEvent_t recorded on `stream` right before the main kernel */
     void *prof_end;             /* optional cudaEvent_t recorded right after it */
+    int debug_withhold_load;    /* testing only, 0 normally: nonzero makes the tensor-core path withhold
+                                   the first x tile of work item 0, so that item's bounded waits run out
+                                   and the call reports SSD_ERR_TIMEOUT through ssd_get_status */
 } ssd_fwd_params;
 
 /* Bytes of device workspace ssd_fwd needs for these parameters (0 on invalid

@@ -53,6 +53,7 @@ class SsdParams(ctypes.Structure):
         ("chunk_len", ctypes.c_int), ("num_seqs", ctypes.c_int), ("io_dtype", ctypes.c_int),
         ("dt_softplus", ctypes.c_int), ("path", ctypes.c_int),
         ("prof_begin", ctypes.c_void_p), ("prof_end", ctypes.c_void_p),
+        ("debug_withhold_load", ctypes.c_int),
     ]
 
 
@@ -100,7 +101,7 @@ def make_params(*, batch, seqlen, nheads, headdim, dstate, ngroups, chunk_len, n
                 prof_end=None) -> SsdParams:
     return SsdParams(int(batch), int(seqlen), int(nheads), int(headdim), int(dstate), int(ngroups),
                      int(chunk_len), int(num_seqs), DTYPES[io_dtype], int(bool(dt_softplus)),
-                     PATHS[path], prof_begin, prof_end)
+                     PATHS[path], prof_begin, prof_end, 0)
 
 
 def workspace_size(params: SsdParams) -> int:

@@ -80,6 +80,7 @@ struct TcParams {
     int *status;
     int H, G, N, heads_per_group;
     int dt_softplus;
+    int withhold_x0;      // testing: work item 0 never loads its first x tile (bounded waits expire)
 };
 
 // --------------------------------------------------------------- smem layout
@@ -96,6 +97,8 @@ struct __align__(1024) TcSmem {
     float dl[kCsd][kQ];                // delta_s (0 on padding rows)
     float w[kCsd][kQ];                 // exp(cs_last - cs_s) * delta_s
     float e[kCsd][kQ];                 // exp(cs_l)
+    float u[kCsd][kQ];                 // exp(cs_{s0} - cs_s) * delta_s, s0 = start of s's 16-column chunk
+    int exact[kCsd];                   // 1: some 16-token chunk decays too fast for the factorised mask
     float alpha[kCsd];                 // exp(cs_last)
     float ldec[kCsd];                  // cs_last (natural log of the block decay)
     uint64_t bc_full[2], bc_empty[2], x_full[2], x_empty[2], cs_full[kCsd], cs_empty[kCsd];
@@ -242,7 +245,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             }
             const float excl = incl - run;
             const float last = __shfl_sync(0xffffffffu, incl, 31);
-            float c2v[4], wv[4], ev[4];
+            float c2v[4], wv[4], ev[4], uv[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const float csn = excl + pre[i];
@@ -250,13 +253,22 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                 wv[i] = ex2_approx((last - csn) * kLog2e) * dl[i];
                 ev[i] = ex2_approx(c2v[i]);
             }
+            // factorised mask: exp2(cs2_l - cs2_s) = exp2(cs2_l - R) * exp2(R - cs2_s) with R the
+            // cs2 of the first token of s's 16-token chunk (lanes 4k..4k+3 hold chunk k)
+            const float Rk = __shfl_sync(0xffffffffu, c2v[0], lane & ~3);
+            const float chunk_end = __shfl_sync(0xffffffffu, c2v[3], lane | 3);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) uv[i] = ex2_approx(Rk - c2v[i]) * dl[i];
+            const int exact = __any_sync(0xffffffffu, Rk - chunk_end > 96.0f) ? 1 : 0;
             *reinterpret_cast<float4 *>(&S.cs2[slot][lane * 4]) = make_float4(c2v[0], c2v[1], c2v[2], c2v[3]);
             *reinterpret_cast<float4 *>(&S.dl[slot][lane * 4]) = make_float4(dl[0], dl[1], dl[2], dl[3]);
             *reinterpret_cast<float4 *>(&S.w[slot][lane * 4]) = make_float4(wv[0], wv[1], wv[2], wv[3]);
             *reinterpret_cast<float4 *>(&S.e[slot][lane * 4]) = make_float4(ev[0], ev[1], ev[2], ev[3]);
+            *reinterpret_cast<float4 *>(&S.u[slot][lane * 4]) = make_float4(uv[0], uv[1], uv[2], uv[3]);
             if (lane == 0) {
                 S.alpha[slot] = ex2_approx(last * kLog2e);
                 S.ldec[slot] = last;
+                S.exact[slot] = exact;
             }
             mbar_arrive(&S.cs_full[slot]);
             if (lane == 0) SSD_TRACE_EV(6, u);
@@ -333,6 +345,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                     const int u = c * KH + j, xs = u & 1;
                     if (u >= 2) ok = mbar_wait(&S.x_empty[xs], ((u >> 1) + 1) & 1, abort);
                     if (!ok) break;
+                    if (prm.withhold_x0 && item_idx == 0 && u == 0) continue;
                     mbar_arrive_expect_tx(&S.x_full[xs], kBoxBytes);
                     tma_load_2d(S.x[xs], &mapX, &S.x_full[xs], (it.h0 + j) * kP, row);
                     issued_x[xs] = u;
@@ -462,43 +475,60 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                     for (int jj = 1; jj < KH; ++jj)
                         if (j == jj) Dh = Dreg[jj];
                     const uint32_t pm_col = tb + lane_base + kColPm + 64 * pi + half * 32;
+                    const bool exact = S.exact[slot] != 0;
 #pragma unroll
                     for (int pair = 0; pair < 2; ++pair) {      // 32 columns -> 16 TMEM columns
                         if (pair < npairs) {                    // warp-uniform
                             const int s0 = s_begin + pair * 32;
+                            uint32_t r[32];
+                            tmem_ld16(tb + lane_base + kColCB + s0, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+                            tmem_ld16(tb + lane_base + kColCB + s0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
+                            float cf[32];                       // column factors
+                            const float R0 = S.cs2[slot][s0], R1 = S.cs2[slot][s0 + 16];
+                            if (!exact) {
+                                const float4 *uu = reinterpret_cast<const float4 *>(&S.u[slot][s0]);
+#pragma unroll
+                                for (int i4 = 0; i4 < 8; ++i4) {
+                                    const float4 v4 = uu[i4];
+                                    cf[4 * i4] = v4.x; cf[4 * i4 + 1] = v4.y;
+                                    cf[4 * i4 + 2] = v4.z; cf[4 * i4 + 3] = v4.w;
+                                }
+                            }
+                            tmem_ld_wait();
+                            if (warp == 7 && lane == 0) SSD_TRACE_EV(19 + pair, u);
+                            if (j == KH - 1 && pair == npairs - 1) {
+                                tc_fence_before();
+                                __syncwarp();
+                                if (lane == 0) mbar_arrive(&S.cb_empty);
+                            }
+                            if (!exact) {
+                                // exp2(cs2_l - cs2_s) delta_s = exp2(cs2_l - R) * exp2(R - cs2_s) delta_s
+                                const float v0 = ex2_approx(rowc - R0), v1 = ex2_approx(rowc - R1);
+#pragma unroll
+                                for (int i = 0; i < 32; ++i) cf[i] *= (i < 16 ? v0 : v1);
+                            } else {
+                                const float4 *cc = reinterpret_cast<const float4 *>(&S.cs2[slot][s0]);
+                                const float4 *dd = reinterpret_cast<const float4 *>(&S.dl[slot][s0]);
+#pragma unroll
+                                for (int i4 = 0; i4 < 8; ++i4) {
+                                    const float4 c4 = cc[i4], d4 = dd[i4];
+                                    cf[4 * i4 + 0] = ex2_approx(rowc - c4.x) * d4.x;
+                                    cf[4 * i4 + 1] = ex2_approx(rowc - c4.y) * d4.y;
+                                    cf[4 * i4 + 2] = ex2_approx(rowc - c4.z) * d4.z;
+                                    cf[4 * i4 + 3] = ex2_approx(rowc - c4.w) * d4.w;
+                                }
+                            }
                             uint32_t packed[16];
 #pragma unroll
-                            for (int sub = 0; sub < 2; ++sub) {
-                                const int s1 = s0 + sub * 16;
-                                uint32_t r[16];
-                                tmem_ld16(tb + lane_base + kColCB + s1, r);
-                                tmem_ld_wait();
-                                if (warp == 7 && lane == 0 && sub == 0) SSD_TRACE_EV(19 + pair, u);
-                                if (j == KH - 1 && pair == npairs - 1 && sub == 1) {
-                                    tc_fence_before();
-                                    __syncwarp();
-                                    if (lane == 0) mbar_arrive(&S.cb_empty);
+                            for (int i2 = 0; i2 < 16; ++i2) {
+                                const int sa = s0 + 2 * i2;
+                                float ma = __uint_as_float(r[2 * i2]) * cf[2 * i2];
+                                float mb = __uint_as_float(r[2 * i2 + 1]) * cf[2 * i2 + 1];
+                                if (sa + 1 >= l) {              // causal edge: s > l is zero, s == l gains D
+                                    ma = sa < l ? ma : (sa == l ? ma + Dh : 0.0f);
+                                    mb = sa + 1 < l ? mb : (sa + 1 == l ? mb + Dh : 0.0f);
                                 }
-                                const float4 *cc = reinterpret_cast<const float4 *>(&S.cs2[slot][s1]);
-                                const float4 *dd = reinterpret_cast<const float4 *>(&S.dl[slot][s1]);
-#pragma unroll
-                                for (int i4 = 0; i4 < 4; ++i4) {
-                                    const float4 c4 = cc[i4], d4 = dd[i4];
-                                    const int sa = s1 + 4 * i4;
-                                    // exponents are differences of the block cumsum (<= 0 for s <= l)
-                                    float m0 = __uint_as_float(r[4 * i4 + 0]) * ex2_approx(rowc - c4.x) * d4.x;
-                                    float m1 = __uint_as_float(r[4 * i4 + 1]) * ex2_approx(rowc - c4.y) * d4.y;
-                                    float m2 = __uint_as_float(r[4 * i4 + 2]) * ex2_approx(rowc - c4.z) * d4.z;
-                                    float m3 = __uint_as_float(r[4 * i4 + 3]) * ex2_approx(rowc - c4.w) * d4.w;
-                                    if (sa + 3 >= l) {          // causal edge: s > l is zero, s == l gains D
-                                        m0 = sa + 0 < l ? m0 : (sa + 0 == l ? m0 + Dh : 0.0f);
-                                        m1 = sa + 1 < l ? m1 : (sa + 1 == l ? m1 + Dh : 0.0f);
-                                        m2 = sa + 2 < l ? m2 : (sa + 2 == l ? m2 + Dh : 0.0f);
-                                        m3 = sa + 3 < l ? m3 : (sa + 3 == l ? m3 + Dh : 0.0f);
-                                    }
-                                    packed[8 * sub + 2 * i4] = pack_bf16x2(m0, m1);
-                                    packed[8 * sub + 2 * i4 + 1] = pack_bf16x2(m2, m3);
-                                }
+                                packed[i2] = pack_bf16x2(ma, mb);
                             }
                             tmem_st16(pm_col + pair * 16, packed);
                         } else {                                // above the diagonal for every row
@@ -634,23 +664,28 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             if (warp == 12 && lane == 0) SSD_TRACE_EV(26, v);
             __nv_bfloat16 *dst = prm.y + ((size_t)tok * prm.H + it.h0 + j) * kP;
 #pragma unroll
-            for (int p0 = 0; p0 < kP; p0 += 16) {
-                uint32_t yd[16];
-                tmem_ld16(tb + lane_base + kColYd + p0, yd);
+            for (int h0 = 0; h0 < kP; h0 += 32) {
+                uint32_t yd[32];
+                tmem_ld16(tb + lane_base + kColYd + h0, *reinterpret_cast<uint32_t(*)[16]>(&yd[0]));
+                tmem_ld16(tb + lane_base + kColYd + h0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&yd[16]));
                 tmem_ld_wait();
-                if (p0 == kP - 16) {
+                if (h0 == kP - 32) {
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&S.yd_empty);
                 }
                 if (t < valid) {
-                    uint32_t pk[8];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        pk[i] = pack_bf16x2(__uint_as_float(yd[2 * i]) + el * __uint_as_float(yo[p0 + 2 * i]),
-                                            __uint_as_float(yd[2 * i + 1]) + el * __uint_as_float(yo[p0 + 2 * i + 1]));
-                    *reinterpret_cast<uint4 *>(dst + p0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    *reinterpret_cast<uint4 *>(dst + p0 + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                    for (int q8 = 0; q8 < 32; q8 += 8) {
+                        uint32_t pk[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int pp = q8 + 2 * i;
+                            pk[i] = pack_bf16x2(__uint_as_float(yd[pp]) + el * __uint_as_float(yo[h0 + pp]),
+                                                __uint_as_float(yd[pp + 1]) + el * __uint_as_float(yo[h0 + pp + 1]));
+                        }
+                        *reinterpret_cast<uint4 *>(dst + h0 + q8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    }
                 }
             }
             __syncwarp();
@@ -678,23 +713,25 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             for (int mt = 0; mt < kMT; ++mt) {
                 const uint32_t hcol = tb + lane_base + kColH + 64 * (j * kMT + mt);
                 const int n = t + 128 * mt;
+                uint32_t r[64];
+#pragma unroll
+                for (int p0 = 0; p0 < kP; p0 += 16)
+                    tmem_ld16(hcol + p0, *reinterpret_cast<uint32_t(*)[16]>(&r[p0]));
+                tmem_ld_wait();
 #pragma unroll
                 for (int p0 = 0; p0 < kP; p0 += 16) {
-                    uint32_t r[16];
-                    tmem_ld16(hcol + p0, r);
-                    tmem_ld_wait();
                     if (!STATE_ONLY && n < N) {
                         uint32_t pk[8];
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
-                            pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+                            pk[i] = pack_bf16x2(__uint_as_float(r[p0 + 2 * i]), __uint_as_float(r[p0 + 2 * i + 1]));
                         *reinterpret_cast<uint4 *>(S.hbf + sw128_offset(n, p0)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                         *reinterpret_cast<uint4 *>(S.hbf + sw128_offset(n, p0 + 8)) =
                             make_uint4(pk[4], pk[5], pk[6], pk[7]);
                     }
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(alpha * __uint_as_float(r[i]));
-                    tmem_st16(hcol + p0, r);
+                    for (int i = 0; i < 16; ++i) r[p0 + i] = __float_as_uint(alpha * __uint_as_float(r[p0 + i]));
+                    tmem_st16(hcol + p0, *reinterpret_cast<uint32_t(*)[16]>(&r[p0]));
                 }
             }
             tmem_st_wait();
@@ -1045,6 +1082,7 @@ cudaError_t launch_tc(const ssd_fwd_params &p, const Plan &plan, const Dims &d, 
     prm.N = p.dstate;
     prm.heads_per_group = d.heads_per_group;
     prm.dt_softplus = p.dt_softplus;
+    prm.withhold_x0 = p.debug_withhold_load != 0;
 
     if (s.segmented) {
         e = launch_walk_any<true>(p.dstate, s.KH, s.max_items, mX, mB, mC, prm, stream);

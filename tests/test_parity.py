@@ -134,6 +134,31 @@ def test_bad_cu_seqlens_reported_in_status():
     assert e.value.code == -5
 
 
+def test_device_wait_timeout_reported():
+    """Failure detection without a fault: work item 0 withholds a tile, its
+    bounded waits run out (about 2 s), the CTA drains, frees TMEM and exits,
+    and the host reads SSD_ERR_TIMEOUT; the context stays usable."""
+    import ctypes
+    import torch
+    import mamba_ssd_layer_fwd_b200 as ssd
+    from _helpers import to_device
+    inp = small_inputs(batch=1, seqlen=512, H=2, P=64, N=64, G=1, Q=256, init=False, seed=12)
+    t = to_device(inp)
+    p = ssd.params_for(t["x"], t["B"], 256, None, True, "tensor")
+    p.debug_withhold_load = 1
+    lib = ssd.library()
+    ws = torch.empty(ssd.workspace_size(p), dtype=torch.uint8, device="cuda")
+    y = torch.empty_like(t["x"])
+    st = torch.cuda.current_stream().cuda_stream or None
+    rc = lib.ssd_fwd(ctypes.byref(p), t["x"].data_ptr(), t["dt"].data_ptr(), t["A_log"].data_ptr(),
+                     t["B"].data_ptr(), t["C"].data_ptr(), t["D"].data_ptr(), None, None, y.data_ptr(), None,
+                     ws.data_ptr(), ws.numel(), st)
+    assert rc == 0
+    assert lib.ssd_get_status(ws.data_ptr(), st) == -4      # SSD_ERR_TIMEOUT
+    # the same context keeps working
+    check_full(inp, path="tensor")
+
+
 # ------------------------------------------------ benchmark shapes, sampled
 
 SAMPLED = {
