@@ -83,6 +83,13 @@ struct TcParams {
     int withhold_x0;      // testing: work item 0 never loads its first x tile (bounded waits expire)
 };
 
+// softplus(v) = max(v, 0) + log1p(exp(-|v|)), out of line: the library log1p is
+// long and the cumsum warp calls it four times per unit.
+__device__ __noinline__ float softplus_f(float v)
+{
+    return fmaxf(v, 0.0f) + log1pf(__expf(-fabsf(v)));
+}
+
 // --------------------------------------------------------------- smem layout
 template <int NST>
 struct __align__(1024) TcSmem {
@@ -232,7 +239,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             for (int i = 0; i < 4; ++i) {
                 const int l = lane * 4 + i;
                 float d = 0.0f;
-                if (l < valid) d = prm.dt_softplus ? fmaxf(r[i], 0.0f) + log1pf(__expf(-fabsf(r[i]))) : r[i];
+                if (l < valid) d = prm.dt_softplus ? softplus_f(r[i]) : r[i];
                 dl[i] = d;
                 run += d * A;
                 pre[i] = run;
@@ -294,7 +301,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                     const uint32_t sW = smem_u32(S.xw[wi]);
 #pragma unroll
                     for (int mt = 0; mt < kMT; ++mt)
-#pragma unroll
+#pragma unroll 1
                         for (int kk = 0; kk < kQ / 16; ++kk)
                             umma_ss(tb + kColH + 64 * (j * kMT + mt),
                                     sdesc_sw128(sB + mt * 32768 + kk * 2048, lbo_m, 1024),
@@ -327,10 +334,10 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                 }
                 for (int j = 0; j < KH; ++j) tma_prefetch_l2_2d(&mapX, (it.h0 + j) * kP, row);
             };
-            for (int c = 0; c < kPrefetch && c < nblk; ++c) prefetch(c);
             for (int c = 0; c < nblk && ok; ++c) {
                 const int bs = c % kSt;
-                if (c + kPrefetch < nblk) prefetch(c + kPrefetch);
+#pragma unroll 1
+                for (int pc = c == 0 ? 0 : c + kPrefetch; pc <= c + kPrefetch && pc < nblk; ++pc) prefetch(pc);
                 if (c >= kSt) ok = mbar_wait(&S.bc_empty[bs], ((c / kSt) + 1) & 1, abort);
                 if (!ok) break;
                 const int row = it.tok0 + c * kQ;
@@ -375,7 +382,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                 tc_fence_after();
                 const uint32_t sC = smem_u32(S.bc[bs][0][0]);
                 const uint32_t sB = smem_u32(S.bc[bs][1][0]);
-#pragma unroll
+#pragma unroll 1
                 for (int kk = 0; kk < NST / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
                     umma_ss(tb + kColCB, sdesc_sw128(sC + off, 16, 1024), sdesc_sw128(sB + off, 16, 1024), id_cb,
@@ -405,7 +412,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                     if (!ok) break;
                     tc_fence_after();
                     const uint32_t sH = smem_u32(S.hbf);
-#pragma unroll
+#pragma unroll 1
                     for (int kk = 0; kk < NST / 16; ++kk) {
                         const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
                         umma_ss(tb + kColYo, sdesc_sw128(sC + off, 16, 1024),
@@ -426,7 +433,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                     if (!ok) break;
                     tc_fence_after();
                     const uint32_t sX = smem_u32(S.x[xs]);
-#pragma unroll
+#pragma unroll 1
                     for (int kk = 0; kk < kQ / 16; ++kk)
                         umma_ts(tb + kColYd, tb + kColPm + 64 * pi + kk * 8,
                                 sdesc_sw128(sX + kk * 2048, 16384, 1024), id_y, kk > 0);
@@ -476,7 +483,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                         if (j == jj) Dh = Dreg[jj];
                     const uint32_t pm_col = tb + lane_base + kColPm + 64 * pi + half * 32;
                     const bool exact = S.exact[slot] != 0;
-#pragma unroll
+#pragma unroll 1
                     for (int pair = 0; pair < 2; ++pair) {      // 32 columns -> 16 TMEM columns
                         if (pair < npairs) {                    // warp-uniform
                             const int s0 = s_begin + pair * 32;
@@ -579,13 +586,17 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             if (!ok) break;
             if (warp == 8 && lane == 0) SSD_TRACE_EV(25, u);
             {
-                // all 16 loads in flight before any math or store
+                // all 16 loads in flight before any math or store.  Step ch of lane i touches the
+                // 16-byte chunk ch ^ (i & 7) of its row: the 8 lanes of each shared-memory phase
+                // then cover 8 different bank groups (the same chunk of 8 rows would be 8-way
+                // conflicted); each chunk is written back to where it was read.
+                const uint32_t rot = (uint32_t)(lane & 7) * 16u;
                 uint4 v[2][8];
 #pragma unroll
                 for (int rr = 0; rr < 2; ++rr)
 #pragma unroll
                     for (int ch = 0; ch < 8; ++ch)
-                        v[rr][ch] = *reinterpret_cast<const uint4 *>(S.x[xs] + (r0 + 32 * rr) * 128 + ch * 16);
+                        v[rr][ch] = *reinterpret_cast<const uint4 *>(S.x[xs] + (r0 + 32 * rr) * 128 + ((ch * 16) ^ rot));
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S.x_empty[xs]);   // X no longer read by this warp
 #pragma unroll
@@ -597,7 +608,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                         __nv_bfloat162 *pv = reinterpret_cast<__nv_bfloat162 *>(&v[rr][ch]);
 #pragma unroll
                         for (int i = 0; i < 4; ++i) pv[i] = __hmul2(pv[i], ws2);
-                        *reinterpret_cast<uint4 *>(S.xw[wi] + t * 128 + ch * 16) = v[rr][ch];   // same swizzled position
+                        *reinterpret_cast<uint4 *>(S.xw[wi] + t * 128 + ((ch * 16) ^ rot)) = v[rr][ch];
                     }
                 }
             }
@@ -694,7 +705,11 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             return true;
         };
 
-        for (int u = 0; u < nunits && ok; ++u) {
+        for (int u = 0; u <= nunits && ok; ++u) {
+            if (u == nunits) {
+                if (!STATE_ONLY && u >= 1) ok = epilogue(u - 1);
+                break;
+            }
             const int c = u / KH, j = u % KH, slot = u % kCsd;
             ok = mbar_wait(&S.cs_full[slot], (u / kCsd) & 1, abort) &&
                  (c == 0 || mbar_wait(&S.h_ready[j], (c - 1) & 1, abort));
@@ -746,7 +761,6 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             if (warp == 12 && lane == 0) SSD_TRACE_EV(10, u);
             if (!STATE_ONLY && u >= 1) ok = epilogue(u - 1);
         }
-        if (!STATE_ONLY && ok && nunits > 0) ok = epilogue(nunits - 1);
         // end of the segment: the state after the last token
         if (ok) {
             for (int j = 0; j < KH; ++j) {

@@ -58,13 +58,11 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete.  Bounded: gives up
-// after `limit_ns` of wall time (or at once when *abort is set), sets *abort
-// and returns false.  No wait in this library can spin forever.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                          uint64_t limit_ns = 2000000000ull)
+// Polling loop of mbar_wait, kept out of line: the kernels have dozens of wait
+// sites, and one shared copy of the loop keeps their instruction footprint
+// (and so instruction-cache misses) small.
+__device__ __noinline__ bool mbar_wait_slow(uint64_t *bar, uint32_t parity, volatile int *abort, uint64_t limit_ns)
 {
-    if (mbar_test(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_test(bar, parity)) return true;
@@ -76,6 +74,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
             }
         }
     }
+}
+
+// Wait for the phase with the given parity to complete.  Bounded: gives up
+// after `limit_ns` of wall time (or at once when *abort is set), sets *abort
+// and returns false.  No wait in this library can spin forever.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                          uint64_t limit_ns = 2000000000ull)
+{
+    if (mbar_test(bar, parity)) return true;
+    return mbar_wait_slow(bar, parity, abort, limit_ns);
 }
 
 // ---------------------------------------------------------------------- TMA
