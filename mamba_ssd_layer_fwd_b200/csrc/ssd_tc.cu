@@ -109,7 +109,7 @@ struct __align__(1024) TcSmem {
     float alpha[kCsd];                 // exp(cs_last)
     float ldec[kCsd];                  // cs_last (natural log of the block decay)
     uint64_t bc_full[2], bc_empty[2], x_full[2], x_empty[2], cs_full[kCsd], cs_empty[kCsd];
-    uint64_t cb_full, cb_empty, pm_full[2], pm_empty[2], hb_full, hb_empty, xw_full[2], xw_empty[2];
+    uint64_t cb_full, cb_empty, pm_full[2], pm_empty[2], hb_full, hb_empty, xw_full[2], xw_empty[2], xw_free[2];
     uint64_t h_ready[2], hs_full[2], y_full, yo_empty, yd_empty, drain_o, drain_s;
     uint32_t tmem_base;
     int abort;
@@ -144,13 +144,17 @@ __device__ long long *g_trace = nullptr;
 template <int NST, int KH, bool STATE_ONLY>
 __global__ void __launch_bounds__(kThreadsTc, 1)
 ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapB,
-            const __grid_constant__ CUtensorMap mapC, const TcParams prm)
+            const __grid_constant__ CUtensorMap mapC, const __grid_constant__ CUtensorMap mapY, const TcParams prm)
 {
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment (128-byte swizzle atoms) computed as an offset from the
     // shared array itself, so every access below stays a shared-memory access
     const uint32_t smem_pad = ((smem_u32(smem_raw) + 1023u) & ~1023u) - smem_u32(smem_raw);
     TcSmem<NST> &S = *reinterpret_cast<TcSmem<NST> *>(smem_raw + smem_pad);
+    // dstate 256 keeps more live registers: there the out-of-line wait call spills,
+    // and the UMMA issue loops run faster unrolled
+    constexpr bool kInlW = NST >= 256;
+    constexpr int kMmaUnroll = NST >= 256 ? 16 : 1;
     const int item_idx = blockIdx.x;
     if (item_idx >= *prm.count) return;
     const TcItem it = prm.items[item_idx];
@@ -164,6 +168,11 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
     const int g = it.h0 / prm.heads_per_group;
     volatile int *abort = &S.abort;
     constexpr int kSt = TcSmem<NST>::kStages, kXwD = TcSmem<NST>::kXw;
+    // Whole 128-token output blocks are staged in the unit's w o X slot (free once the
+    // state UMMA has read it) and written by TMA stores, one 32-row slab per epilogue
+    // warp: coalesced full-line writes instead of 16-byte pieces of 32 rows.  Needs
+    // two w o X slots, so the next unit's w o X pass runs meanwhile.
+    constexpr bool kTmaY = !STATE_ONLY && kXwD >= 2;
     constexpr int kMT = NST >= 256 ? 2 : 1;        // 128-row state tiles per head (H^T rows = n)
 
     if (tid == 0) {
@@ -173,7 +182,8 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             mbar_init(&S.x_full[i], 1);
             mbar_init(&S.x_empty[i], STATE_ONLY ? 2 : 3);     // w o X warps (+ output issuer)
             mbar_init(&S.xw_full[i], 2);
-            mbar_init(&S.xw_empty[i], 1);
+            mbar_init(&S.xw_empty[i], kTmaY ? 4 : 1);       // epilogue warps, else the state issuer
+            mbar_init(&S.xw_free[i], 1);
             mbar_init(&S.pm_full[i], kMaskWarps);
             mbar_init(&S.pm_empty[i], 1);
             mbar_init(&S.h_ready[i], 1);
@@ -230,7 +240,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
 #pragma unroll
             for (int jj = 1; jj < KH; ++jj)
                 if (j == jj) A = Areg[jj];
-            if (u >= kCsd) ok = mbar_wait(&S.cs_empty[slot], ((u / kCsd) + 1) & 1, abort);
+            if (u >= kCsd) ok = mbar_wait<kInlW>(&S.cs_empty[slot], ((u / kCsd) + 1) & 1, abort);
             if (!ok) break;
             // lane owns tokens 4*lane .. 4*lane+3
             float dl[4], pre[4];
@@ -289,31 +299,31 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             bool ok = true;
             for (int c = 0; c < nblk && ok; ++c) {
                 const int bs = c % kSt;
-                ok = mbar_wait(&S.bc_full[bs], (c / kSt) & 1, abort);
+                ok = mbar_wait<kInlW>(&S.bc_full[bs], (c / kSt) & 1, abort);
                 if (!ok) break;
                 const uint32_t sB = smem_u32(S.bc[bs][1][0]);
                 for (int j = 0; j < KH && ok; ++j) {
                     const int u = c * KH + j, wi = u % kXwD;
-                    ok = mbar_wait(&S.xw_full[wi], (u / kXwD) & 1, abort) && mbar_wait(&S.hs_full[j], c & 1, abort);
+                    ok = mbar_wait<kInlW>(&S.xw_full[wi], (u / kXwD) & 1, abort) && mbar_wait<kInlW>(&S.hs_full[j], c & 1, abort);
                     SSD_TRACE_EV(15, u);
                     if (!ok) break;
                     tc_fence_after();
                     const uint32_t sW = smem_u32(S.xw[wi]);
 #pragma unroll
                     for (int mt = 0; mt < kMT; ++mt)
-#pragma unroll 1
+#pragma unroll kMmaUnroll
                         for (int kk = 0; kk < kQ / 16; ++kk)
                             umma_ss(tb + kColH + 64 * (j * kMT + mt),
                                     sdesc_sw128(sB + mt * 32768 + kk * 2048, lbo_m, 1024),
                                     sdesc_sw128(sW + kk * 2048, 16384, 1024), id_h, 1);
-                    umma_commit(&S.xw_empty[wi]);
+                    umma_commit(kTmaY ? &S.xw_free[wi] : &S.xw_empty[wi]);
                     umma_commit(&S.h_ready[j]);
                     SSD_TRACE_EV(4, u);
                 }
                 umma_commit(&S.bc_empty[bs]);
             }
             umma_commit(&S.drain_s);
-            mbar_wait(&S.drain_s, 0, abort, 200000000ull);
+            mbar_wait<kInlW>(&S.drain_s, 0, abort, 200000000ull);
         }
     } else if (warp == 2) {
         // ------------------------------------------------------ TMA producer
@@ -338,7 +348,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                 const int bs = c % kSt;
 #pragma unroll 1
                 for (int pc = c == 0 ? 0 : c + kPrefetch; pc <= c + kPrefetch && pc < nblk; ++pc) prefetch(pc);
-                if (c >= kSt) ok = mbar_wait(&S.bc_empty[bs], ((c / kSt) + 1) & 1, abort);
+                if (c >= kSt) ok = mbar_wait<kInlW>(&S.bc_empty[bs], ((c / kSt) + 1) & 1, abort);
                 if (!ok) break;
                 const int row = it.tok0 + c * kQ;
                 mbar_arrive_expect_tx(&S.bc_full[bs], kBcBytes);
@@ -350,7 +360,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                 SSD_TRACE_EV(0, c);
                 for (int j = 0; j < KH; ++j) {
                     const int u = c * KH + j, xs = u & 1;
-                    if (u >= 2) ok = mbar_wait(&S.x_empty[xs], ((u >> 1) + 1) & 1, abort);
+                    if (u >= 2) ok = mbar_wait<kInlW>(&S.x_empty[xs], ((u >> 1) + 1) & 1, abort);
                     if (!ok) break;
                     if (prm.withhold_x0 && item_idx == 0 && u == 0) continue;
                     mbar_arrive_expect_tx(&S.x_full[xs], kBoxBytes);
@@ -363,8 +373,8 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                 // drain: wait (bounded) for copies still in flight before the CTA exits
                 for (int i = 0; i < 2; ++i) {
                     if (i < kSt && issued_bc[i] >= 0)
-                        mbar_wait(&S.bc_full[i], (issued_bc[i] / kSt) & 1, abort, 200000000ull);
-                    if (issued_x[i] >= 0) mbar_wait(&S.x_full[i], (issued_x[i] >> 1) & 1, abort, 200000000ull);
+                        mbar_wait<kInlW>(&S.bc_full[i], (issued_bc[i] / kSt) & 1, abort, 200000000ull);
+                    if (issued_x[i] >= 0) mbar_wait<kInlW>(&S.x_full[i], (issued_x[i] >> 1) & 1, abort, 200000000ull);
                 }
             }
         }
@@ -377,12 +387,12 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             // CB = C_c B_c^T into the single CB accumulator
             auto issue_cb = [&](int c) -> bool {
                 const int bs = c % kSt;
-                if (!mbar_wait(&S.bc_full[bs], (c / kSt) & 1, abort)) return false;
-                if (c >= 1 && !mbar_wait(&S.cb_empty, (c - 1) & 1, abort)) return false;
+                if (!mbar_wait<kInlW>(&S.bc_full[bs], (c / kSt) & 1, abort)) return false;
+                if (c >= 1 && !mbar_wait<kInlW>(&S.cb_empty, (c - 1) & 1, abort)) return false;
                 tc_fence_after();
                 const uint32_t sC = smem_u32(S.bc[bs][0][0]);
                 const uint32_t sB = smem_u32(S.bc[bs][1][0]);
-#pragma unroll 1
+#pragma unroll kMmaUnroll
                 for (int kk = 0; kk < NST / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
                     umma_ss(tb + kColCB, sdesc_sw128(sC + off, 16, 1024), sdesc_sw128(sB + off, 16, 1024), id_cb,
@@ -405,14 +415,14 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                 for (int j = 0; j < KH && ok; ++j) {
                     const int u = c * KH + j, xs = u & 1, pi = u & 1;
                     // Yo = C Hbf^T
-                    ok = mbar_wait(&S.hb_full, u & 1, abort);
+                    ok = mbar_wait<kInlW>(&S.hb_full, u & 1, abort);
                     SSD_TRACE_EV(14, u);
-                    ok = ok && (u == 0 || mbar_wait(&S.yo_empty, (u - 1) & 1, abort));
+                    ok = ok && (u == 0 || mbar_wait<kInlW>(&S.yo_empty, (u - 1) & 1, abort));
                     SSD_TRACE_EV(17, u);
                     if (!ok) break;
                     tc_fence_after();
                     const uint32_t sH = smem_u32(S.hbf);
-#pragma unroll 1
+#pragma unroll kMmaUnroll
                     for (int kk = 0; kk < NST / 16; ++kk) {
                         const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
                         umma_ss(tb + kColYo, sdesc_sw128(sC + off, 16, 1024),
@@ -426,14 +436,14 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                         if (!ok) break;
                     }
                     // Yd = Pm X
-                    ok = mbar_wait(&S.pm_full[pi], (u >> 1) & 1, abort) &&
-                         mbar_wait(&S.x_full[xs], (u >> 1) & 1, abort) &&
-                         (u == 0 || mbar_wait(&S.yd_empty, (u - 1) & 1, abort));
+                    ok = mbar_wait<kInlW>(&S.pm_full[pi], (u >> 1) & 1, abort) &&
+                         mbar_wait<kInlW>(&S.x_full[xs], (u >> 1) & 1, abort) &&
+                         (u == 0 || mbar_wait<kInlW>(&S.yd_empty, (u - 1) & 1, abort));
                     SSD_TRACE_EV(16, u);
                     if (!ok) break;
                     tc_fence_after();
                     const uint32_t sX = smem_u32(S.x[xs]);
-#pragma unroll 1
+#pragma unroll kMmaUnroll
                     for (int kk = 0; kk < kQ / 16; ++kk)
                         umma_ts(tb + kColYd, tb + kColPm + 64 * pi + kk * 8,
                                 sdesc_sw128(sX + kk * 2048, 16384, 1024), id_y, kk > 0);
@@ -446,7 +456,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             }
             // every UMMA issued so far has completed before TMEM is released
             umma_commit(&S.drain_o);
-            mbar_wait(&S.drain_o, 0, abort, 200000000ull);
+            mbar_wait<kInlW>(&S.drain_o, 0, abort, 200000000ull);
         }
     } else if ((warp >= 4 && warp < 8) || warp == 10 || warp == 11) {
         // ------------------------------------------------------------- mask
@@ -465,13 +475,13 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             for (int j = 0; j < KH; ++j) Dreg[j] = prm.D ? prm.D[it.h0 + j] : 0.0f;
             bool ok = true;
             for (int c = 0; c < nblk && ok; ++c) {
-                ok = mbar_wait(&S.cb_full, c & 1, abort);
+                ok = mbar_wait<kInlW>(&S.cb_full, c & 1, abort);
                 if (!ok) break;
                 tc_fence_after();
                 for (int j = 0; j < KH; ++j) {
                     const int u = c * KH + j, slot = u % kCsd, pi = u & 1;
-                    ok = mbar_wait(&S.cs_full[slot], (u / kCsd) & 1, abort) &&
-                         (u < 2 || mbar_wait(&S.pm_empty[pi], ((u >> 1) + 1) & 1, abort));
+                    ok = mbar_wait<kInlW>(&S.cs_full[slot], (u / kCsd) & 1, abort) &&
+                         (u < 2 || mbar_wait<kInlW>(&S.pm_empty[pi], ((u >> 1) + 1) & 1, abort));
                     if (!ok) break;
                     tc_fence_after();
                     if (warp == 4 && lane == 0) SSD_TRACE_EV(7, u);
@@ -580,9 +590,9 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
         const int r0 = (warp - 8) * 64 + lane;          // rows r0 and r0 + 32
         for (int u = 0; u < nunits && ok; ++u) {
             const int slot = u % kCsd, xs = u & 1, wi = u % kXwD;
-            ok = mbar_wait(&S.cs_full[slot], (u / kCsd) & 1, abort) &&
-                 mbar_wait(&S.x_full[xs], (u >> 1) & 1, abort) &&
-                 (u < kXwD || mbar_wait(&S.xw_empty[wi], ((u / kXwD) + 1) & 1, abort));
+            ok = mbar_wait<kInlW>(&S.cs_full[slot], (u / kCsd) & 1, abort) &&
+                 mbar_wait<kInlW>(&S.x_full[xs], (u >> 1) & 1, abort) &&
+                 (u < kXwD || mbar_wait<kInlW>(&S.xw_empty[wi], ((u / kXwD) + 1) & 1, abort));
             if (!ok) break;
             if (warp == 8 && lane == 0) SSD_TRACE_EV(25, u);
             {
@@ -649,6 +659,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             }
         }
         tmem_st_wait();
+        if (kTmaY && lane == 0) tma_prefetch_desc(&mapY);
         bool ok = true;
         float ldec_sum[KH];
 #pragma unroll
@@ -657,7 +668,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
         // epilogue of unit v: y = Yd + exp(cs_l) Yo for this thread's row
         auto epilogue = [&](int v) -> bool {
             const int c = v / KH, j = v % KH, slot = v % kCsd;
-            if (!mbar_wait(&S.y_full, v & 1, abort)) return false;
+            if (!mbar_wait<kInlW>(&S.y_full, v & 1, abort)) return false;
             tc_fence_after();
             if (warp == 12 && lane == 0) SSD_TRACE_EV(12, v);
             const int valid = min(kQ, it.len - c * kQ);
@@ -674,6 +685,11 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             if (lane == 0) mbar_arrive(&S.yo_empty);
             if (warp == 12 && lane == 0) SSD_TRACE_EV(26, v);
             __nv_bfloat16 *dst = prm.y + ((size_t)tok * prm.H + it.h0 + j) * kP;
+            const int wi = v % kXwD;
+            uint8_t *stage = S.xw[wi] + q * 32 * 128;     // this warp's 32 rows, 128-byte swizzled
+            const bool via_tma = kTmaY && valid == kQ;
+            // the slot's w o X tile is free once the state UMMA of unit v has completed
+            if (kTmaY && !mbar_wait<kInlW>(&S.xw_free[wi], (v / kXwD) & 1, abort)) return false;
 #pragma unroll
             for (int h0 = 0; h0 < kP; h0 += 32) {
                 uint32_t yd[32];
@@ -685,7 +701,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&S.yd_empty);
                 }
-                if (t < valid) {
+                if (via_tma || t < valid) {
 #pragma unroll
                     for (int q8 = 0; q8 < 32; q8 += 8) {
                         uint32_t pk[4];
@@ -695,12 +711,25 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                             pk[i] = pack_bf16x2(__uint_as_float(yd[pp]) + el * __uint_as_float(yo[h0 + pp]),
                                                 __uint_as_float(yd[pp + 1]) + el * __uint_as_float(yo[h0 + pp + 1]));
                         }
-                        *reinterpret_cast<uint4 *>(dst + h0 + q8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        const uint4 v4 = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        if (via_tma)
+                            *reinterpret_cast<uint4 *>(stage + sw128_offset(lane, h0 + q8)) = v4;
+                        else
+                            *reinterpret_cast<uint4 *>(dst + h0 + q8) = v4;
                     }
                 }
             }
+            if (via_tma) fence_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&S.cs_empty[slot]);
+            if (lane == 0) {
+                if (via_tma) {
+                    tma_store_2d(&mapY, stage, (it.h0 + j) * kP, it.tok0 + c * kQ + q * 32);
+                    bulk_commit();
+                    bulk_wait_read_all();
+                }
+                if (kTmaY) mbar_arrive(&S.xw_empty[wi]);
+                mbar_arrive(&S.cs_empty[slot]);
+            }
             if (warp == 12 && lane == 0) SSD_TRACE_EV(13, v);
             return true;
         };
@@ -711,10 +740,10 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                 break;
             }
             const int c = u / KH, j = u % KH, slot = u % kCsd;
-            ok = mbar_wait(&S.cs_full[slot], (u / kCsd) & 1, abort) &&
-                 (c == 0 || mbar_wait(&S.h_ready[j], (c - 1) & 1, abort));
+            ok = mbar_wait<kInlW>(&S.cs_full[slot], (u / kCsd) & 1, abort) &&
+                 (c == 0 || mbar_wait<kInlW>(&S.h_ready[j], (c - 1) & 1, abort));
             if (!ok) break;
-            if (!STATE_ONLY) ok = (u == 0 || mbar_wait(&S.hb_empty, (u - 1) & 1, abort));
+            if (!STATE_ONLY) ok = (u == 0 || mbar_wait<kInlW>(&S.hb_empty, (u - 1) & 1, abort));
             if (!ok) break;
             tc_fence_after();
             if (warp == 12 && lane == 0) SSD_TRACE_EV(9, u);
@@ -764,7 +793,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
         // end of the segment: the state after the last token
         if (ok) {
             for (int j = 0; j < KH; ++j) {
-                ok = mbar_wait(&S.h_ready[j], (nblk - 1) & 1, abort);
+                ok = mbar_wait<kInlW>(&S.h_ready[j], (nblk - 1) & 1, abort);
                 if (!ok) break;
                 tc_fence_after();
                 const int h = it.h0 + j;
@@ -791,6 +820,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                 if (STATE_ONLY && t == 0) prm.seglogdec[(size_t)it.gseg * prm.H + h] = ldec_sum[j];
             }
         }
+        if (kTmaY && lane == 0) bulk_wait_all();       // this warp's y stores have landed
     }
 
     // ------------------------------------------------------------ teardown
@@ -913,11 +943,27 @@ tc_seg_scan_kernel(const TcItem *__restrict__ items, const int *__restrict__ cou
     const int e = blockIdx.z * 256 + threadIdx.x;
     if (e >= PN) return;
     float hv = init ? init[((size_t)it.seq * H + h) * PN + e] : 0.0f;
-    for (int k = 0; k < it.nseg; ++k) {
-        const size_t o = ((size_t)(gs + k) * H + h) * PN + e;
-        const float sv = k < it.nseg - 1 ? segstate[o] : 0.0f;
-        segstate[o] = hv;
-        if (k < it.nseg - 1) hv = fmaf(__expf(seglogdec[(size_t)(gs + k) * H + h]), hv, sv);
+    // segment k's slot holds the state measured over segment k from zero on entry and
+    // the state entering segment k on exit; loads go out in groups so that the chain
+    // waits on memory once per group, not once per segment
+    constexpr int kGroup = 8;
+    for (int k0 = 0; k0 < it.nseg; k0 += kGroup) {
+        float sv[kGroup], dk[kGroup];
+#pragma unroll
+        for (int i = 0; i < kGroup; ++i) {
+            const int k = k0 + i;
+            const bool has = k < it.nseg - 1;
+            sv[i] = has ? segstate[((size_t)(gs + k) * H + h) * PN + e] : 0.0f;
+            dk[i] = has ? __expf(seglogdec[(size_t)(gs + k) * H + h]) : 0.0f;
+        }
+#pragma unroll
+        for (int i = 0; i < kGroup; ++i) {
+            const int k = k0 + i;
+            if (k < it.nseg) {
+                segstate[((size_t)(gs + k) * H + h) * PN + e] = hv;
+                hv = fmaf(dk[i], hv, sv[i]);
+            }
+        }
     }
 }
 
@@ -935,14 +981,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
     return fn;
 }
 
-// 2-D bf16 view [rows][inner] with a {64, 128} box and 128-byte swizzle.
-bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows)
+// 2-D bf16 view [rows][inner] with a {64, box_rows} box and 128-byte swizzle.
+bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, uint32_t box_rows = 128)
 {
     auto enc = encode_fn();
     if (!enc) return false;
     cuuint64_t dims[2] = {inner, rows};
     cuuint64_t strides[1] = {inner * 2};
-    cuuint32_t box[2] = {64, 128};
+    cuuint32_t box[2] = {64, box_rows};
     cuuint32_t es[2] = {1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -954,17 +1000,9 @@ struct TcPlanShape {
     bool segmented;
 };
 
-int sm_count()
-{
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
-    return n;
-}
+// The work split is a pure function of the parameters (the workspace size must
+// not depend on which GPU answers), sized for the B200's 148 SMs.
+constexpr int kPlanSMs = 148;
 
 TcPlanShape plan_shape(const ssd_fwd_params &p)
 {
@@ -975,16 +1013,35 @@ TcPlanShape plan_shape(const ssd_fwd_params &p)
     s.n_hb = p.nheads / s.KH;
     const int nseq = p.num_seqs > 0 ? p.num_seqs : p.batch;
     const long long tokens = (long long)p.batch * p.seqlen;
-    const int target = 2 * 148;                       // work items wanted (two per SM)
+    const int target = 2 * kPlanSMs;                  // work items wanted (two per SM)
     long long seg;
     if (p.num_seqs > 0) {
         // packed: bound the longest item so no sequence dominates the makespan
         seg = (tokens * s.n_hb + target - 1) / target;
         seg = seg < 1024 ? 1024 : seg;
     } else {
+        // equal-length sequences: pick the segment count with the smallest modelled
+        // makespan, in 128-token block steps of one SM.  Pass 2 runs
+        // ceil(pairs * n / SMs) rounds of items of ceil(blocks / n) blocks; pass 1
+        // (state only, about 0.65 of a pass-2 block) the same over n - 1 segments;
+        // each round costs about 1.5 blocks of fill and drain, the segment scan 2.
         const long long pairs = (long long)p.batch * s.n_hb;
-        long long nseg = pairs >= 148 ? 1 : (target + pairs - 1) / pairs;
-        seg = (p.seqlen + nseg - 1) / (nseg > 0 ? nseg : 1);
+        const long long nblk = (p.seqlen + kQ - 1) / kQ;
+        const long long sms = kPlanSMs;
+        long long best_n = 1;
+        double best = 1e300;
+        for (long long n = 1; n <= 64 && n <= nblk; ++n) {
+            const long long bps = (nblk + n - 1) / n;
+            const long long r2 = (pairs * n + sms - 1) / sms;
+            const long long r1 = n > 1 ? (pairs * (n - 1) + sms - 1) / sms : 0;
+            const double cost = (double)bps * ((double)r2 + 0.65 * (double)r1) + 1.5 * (double)(r1 + r2) +
+                                (n > 1 ? 2.0 : 0.0);
+            if (cost < best - 1e-9) {
+                best = cost;
+                best_n = n;
+            }
+        }
+        seg = (nblk + best_n - 1) / best_n * kQ;
     }
     seg = (seg + kQ - 1) / kQ * kQ;
     if (seg < kQ) seg = kQ;
@@ -1000,31 +1057,33 @@ TcPlanShape plan_shape(const ssd_fwd_params &p)
 
 template <int NST, int KH, bool SO>
 cudaError_t launch_walk(int grid, const CUtensorMap &mX, const CUtensorMap &mB, const CUtensorMap &mC,
+                        const CUtensorMap &mY,
                         const TcParams &prm, cudaStream_t st)
 {
     const size_t smem = tc_smem_bytes<NST>();
     cudaError_t e = cudaFuncSetAttribute(ssd_tc_walk<NST, KH, SO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    ssd_tc_walk<NST, KH, SO><<<grid, kThreadsTc, smem, st>>>(mX, mB, mC, prm);
+    ssd_tc_walk<NST, KH, SO><<<grid, kThreadsTc, smem, st>>>(mX, mB, mC, mY, prm);
     return cudaGetLastError();
 }
 
 template <int NST, bool SO>
 cudaError_t launch_walk_kh(int KH, int grid, const CUtensorMap &mX, const CUtensorMap &mB, const CUtensorMap &mC,
+                           const CUtensorMap &mY,
                            const TcParams &prm, cudaStream_t st)
 {
-    return KH == 2 ? launch_walk<NST, 2, SO>(grid, mX, mB, mC, prm, st)
-                   : launch_walk<NST, 1, SO>(grid, mX, mB, mC, prm, st);
+    return KH == 2 ? launch_walk<NST, 2, SO>(grid, mX, mB, mC, mY, prm, st)
+                   : launch_walk<NST, 1, SO>(grid, mX, mB, mC, mY, prm, st);
 }
 
 template <bool SO>
 cudaError_t launch_walk_any(int N, int KH, int grid, const CUtensorMap &mX, const CUtensorMap &mB,
-                            const CUtensorMap &mC, const TcParams &prm, cudaStream_t st)
+                            const CUtensorMap &mC, const CUtensorMap &mY, const TcParams &prm, cudaStream_t st)
 {
-    if (N == 256) return launch_walk<256, 1, SO>(grid, mX, mB, mC, prm, st);
-    return N == 128 ? launch_walk_kh<128, SO>(KH, grid, mX, mB, mC, prm, st)
-                    : launch_walk_kh<64, SO>(KH, grid, mX, mB, mC, prm, st);
+    if (N == 256) return launch_walk<256, 1, SO>(grid, mX, mB, mC, mY, prm, st);
+    return N == 128 ? launch_walk_kh<128, SO>(KH, grid, mX, mB, mC, mY, prm, st)
+                    : launch_walk_kh<64, SO>(KH, grid, mX, mB, mC, mY, prm, st);
 }
 
 size_t align256(size_t v) { return (v + 255) / 256 * 256; }
@@ -1073,8 +1132,10 @@ cudaError_t launch_tc(const ssd_fwd_params &p, const Plan &plan, const Dims &d, 
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || tokens == 0) return e;
 
-    CUtensorMap mX, mB, mC;
+    CUtensorMap mX, mB, mC, mY;
+    // y has x's layout; its map moves 32-row slabs (one per epilogue warp)
     if (!make_map(&mX, a.x, (uint64_t)p.nheads * kP, (uint64_t)tokens) ||
+        !make_map(&mY, a.y, (uint64_t)p.nheads * kP, (uint64_t)tokens, 32) ||
         !make_map(&mB, a.B, (uint64_t)p.ngroups * p.dstate, (uint64_t)tokens) ||
         !make_map(&mC, a.C, (uint64_t)p.ngroups * p.dstate, (uint64_t)tokens))
         return cudaErrorInvalidValue;
@@ -1099,7 +1160,7 @@ cudaError_t launch_tc(const ssd_fwd_params &p, const Plan &plan, const Dims &d, 
     prm.withhold_x0 = p.debug_withhold_load != 0;
 
     if (s.segmented) {
-        e = launch_walk_any<true>(p.dstate, s.KH, s.max_items, mX, mB, mC, prm, stream);
+        e = launch_walk_any<true>(p.dstate, s.KH, s.max_items, mX, mB, mC, mY, prm, stream);
         if (e != cudaSuccess) return e;
         const dim3 gs(s.max_segments, p.nheads, (PN + 255) / 256);
         tc_seg_scan_kernel<<<gs, 256, 0, stream>>>(items, plan.count, s.n_hb, 0, segstate, seglogdec, a.init,
@@ -1107,7 +1168,7 @@ cudaError_t launch_tc(const ssd_fwd_params &p, const Plan &plan, const Dims &d, 
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (prof_begin) cudaEventRecord(prof_begin, stream);
-    e = launch_walk_any<false>(p.dstate, s.KH, s.max_items, mX, mB, mC, prm, stream);
+    e = launch_walk_any<false>(p.dstate, s.KH, s.max_items, mX, mB, mC, mY, prm, stream);
     if (prof_end) cudaEventRecord(prof_end, stream);
     return e;
 }

@@ -79,11 +79,25 @@ __device__ __noinline__ bool mbar_wait_slow(uint64_t *bar, uint32_t parity, vola
 // Wait for the phase with the given parity to complete.  Bounded: gives up
 // after `limit_ns` of wall time (or at once when *abort is set), sets *abort
 // and returns false.  No wait in this library can spin forever.
+// kInline expands the polling loop at the call site instead (better where
+// register pressure makes the out-of-line call spill).
+template <bool kInline = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
                                           uint64_t limit_ns = 2000000000ull)
 {
     if (mbar_test(bar, parity)) return true;
-    return mbar_wait_slow(bar, parity, abort, limit_ns);
+    if (!kInline) return mbar_wait_slow(bar, parity, abort, limit_ns);
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_test(bar, parity)) return true;
+        if ((it & 255u) == 0) {
+            if (*abort) return false;
+            if (globaltimer_ns() - t0 > limit_ns) {
+                *abort = 1;
+                return false;
+            }
+        }
+    }
 }
 
 // ---------------------------------------------------------------------- TMA
@@ -95,6 +109,21 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, u
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
         : "memory");
 }
+
+// Tile store shared -> global (bulk-group completion, no multicast).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int c0, int c1)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(smem_u32(src)), "r"(c0), "r"(c1)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Shared-memory sources of this thread's committed bulk stores have been read.
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// This thread's committed bulk stores are complete.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // Bring a tile into L2 ahead of its load (no shared memory, no completion).
 __device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *map, int c0, int c1)
