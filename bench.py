@@ -238,7 +238,7 @@ def run_reference(args):
             per_step.append(rate)
     value = float(statistics.median(per_step))
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "impl": "reference", "metric": DECODE_METRIC if args.op == "decode" else METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000.0 * tokens / value, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
@@ -390,6 +390,140 @@ def run_ours(args):
     return 0
 
 
+DECODE_METRIC = "SSD decode step tokens/s at 1 B200; % of HBM roofline"
+
+
+def decode_bytes(inp: dict) -> int:
+    """Compulsory traffic of one decoding step: the fp32 state read and
+    written, plus x, y, dt, B, C of the new token."""
+    x, B = inp["x"], inp["B"]
+    b, H, P = x.shape[0], x.shape[2], x.shape[3]
+    G, N = B.shape[2], B.shape[3]
+    es = 2 if inp["io_dtype"] == "bf16" else 4
+    return int(2 * b * H * P * N * 4 + (2 * b * H * P + b * H + 2 * b * G * N) * es)
+
+
+def run_decode(args):
+    """One `ssd_decode_step` per step over every row of the decode workload
+    (the state stays resident on the device, as in serving)."""
+    import torch
+    import torch.distributed as dist
+    import mamba_ssd_layer_fwd_b200 as ssd
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    inp = ssd_inputs.make_inputs(ssd_inputs.workload(args.workload), seed=args.seed)
+    if inp["x"].shape[1] != 1:
+        raise SystemExit("--op decode needs a one-token workload (decode_2p7b)")
+    io = torch.bfloat16 if inp["io_dtype"] == "bf16" else torch.float32
+    host = {k: torch.from_numpy(np.ascontiguousarray(inp[k][:, 0])).to(io).pin_memory()
+            for k in ("x", "dt", "B", "C")}
+    d = {k: v.to(dev) for k, v in host.items()}
+    A_log = torch.from_numpy(inp["A_log"]).to(dev)
+    D = torch.from_numpy(inp["D"]).to(dev)
+    state = torch.from_numpy(inp["initial_states"]).to(dev)
+    y = torch.empty_like(d["x"])
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ssd.ssd_decode_step(d["x"], d["dt"], A_log, d["B"], d["C"], D, state, y=y, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    for row in ev:
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.current_device() if world == 1 else local)
+    if rank == 0:
+        sampler.start()
+        time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    for i in range(K):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    wall = time.perf_counter() - wall0
+    clocks = sampler.stop() if rank == 0 else None
+    ms = max_over_ranks([statistics.mean(ev[i][0].elapsed_time(ev[i][1]) for i in range(K))], dev)[0]
+
+    # end to end: the new token's inputs from pinned host memory, y back to the host
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = y_host.numel() * y_host.element_size()
+    e2e_ms = []
+    for i in range(args.warmup + K):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        flush.zero_()
+        e0.record(stream)
+        for k, v in host.items():
+            d[k].copy_(v, non_blocking=True)
+        step()
+        y_host.copy_(y, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(e0.elapsed_time(e1))
+    e2e = max_over_ranks([statistics.mean(e2e_ms)], dev)[0]
+
+    rows = inp["x"].shape[0]
+    value = whole_job_throughput(rows, world, ms)
+    nbytes = decode_bytes(inp)
+    peak, peak_kind = measured_peaks()
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            rate, cores, desc, _ = cpu_oracle_rate(inp, budget_s=args.ref_seconds)
+            cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc}
+        w = inp["workload"]
+        line = {
+            "metric": DECODE_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": inp["io_dtype"],
+            "data": "synthetic (seeded generator, value distributions of the workload)",
+            "config": {"workload": w.name, "rows": rows, "nheads": w.nheads, "headdim": w.headdim,
+                       "dstate": w.dstate, "ngroups": w.ngroups, "io_dtype": w.io_dtype,
+                       "state": "fp32, resident, updated in place",
+                       "parallelism": f"replicas x{world}" if world > 1 else "1 gpu",
+                       "l2": "flushed before every timed step (512 MiB write)"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None, "kernel": "ssd_decode_kernel",
+                         "kernel_ms": ms, "alg_bytes": nbytes,
+                         "peak_source": f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"},
+            "cpu_baseline": cpu,
+            "e2e": {"value": whole_job_throughput(rows, world, e2e), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": K,
+            "clocks": clocks,
+            "wall_s_timed_region": wall,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -401,10 +535,16 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--ref-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", choices=["fwd", "decode"], default="fwd",
+                    help="fwd: the chunked forward (default); decode: one recurrent step per row")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)      # at least 3 untimed warm-up steps
+    if args.op == "decode" and args.workload == "mamba2_2p7b":
+        args.workload = "decode_2p7b"
     if args.impl == "reference":
         return run_reference(args)
+    if args.op == "decode":
+        return run_decode(args)
     return run_ours(args)
 
 

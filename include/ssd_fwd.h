@@ -145,6 +145,40 @@ SSD_API ssd_status ssd_fwd_noalloc(const ssd_fwd_params *p,
                    const float *initial_states, const int32_t *cu_seqlens,
                    void *y, float *final_states, void *stream, int sync_status);
 
+/* One decoding step: the recurrent (linear) mode of the same layer
+ * ("Transformers are SSMs", Sec. 3.4.1 eq. (8)) applied to a single new token
+ * of every row, with the state carried in place between calls:
+ *
+ *     delta = softplus(dt[b, h])  (dt itself when dt_softplus == 0)
+ *     a     = exp(delta * -exp(A_log[h]))
+ *     state[b, h] <- a * state[b, h] + (delta * x[b, h, :]) (outer) B[b, g, :]
+ *     y[b, h, :]   = state[b, h] @ C[b, g, :] + D[h] * x[b, h, :]
+ *
+ * A prefill with ssd_fwd(..., final_states) followed by steps from that state
+ * reproduces ssd_fwd over the concatenated tokens.
+ * Layouts (row-major, contiguous): x, y (batch, nheads, headdim) and
+ * dt (batch, nheads) in io dtype; B, C (batch, ngroups, dstate) io dtype;
+ * A_log, D (nheads) float32; state (batch, nheads, headdim, dstate) float32,
+ * read and overwritten.  B, C and state must be 16-byte aligned; x, dt, y
+ * naturally aligned.  D may be NULL (0).  All pointers are caller-owned device
+ * pointers; no workspace, nothing allocated, asynchronous on `stream`.
+ * Returns SSD_ERR_INVALID_ARG (bad dimension or pointer), SSD_ERR_UNSUPPORTED
+ * (dstate not a multiple of 4 or above 256), SSD_ERR_CUDA (launch failed). */
+typedef struct ssd_step_params {
+    int batch;                  /* rows >= 0 (0: nothing to do) */
+    int nheads;                 /* H >= 1 */
+    int headdim;                /* P >= 1 */
+    int dstate;                 /* N: multiple of 4, <= 256 */
+    int ngroups;                /* G >= 1, nheads % ngroups == 0 */
+    ssd_dtype io_dtype;
+    int dt_softplus;            /* 1: delta = softplus(dt); 0: delta = dt */
+} ssd_step_params;
+
+SSD_API ssd_status ssd_decode_step(const ssd_step_params *p,
+                   const void *x, const void *dt, const float *A_log,
+                   const void *B, const void *C, const float *D,
+                   float *state, void *y, void *stream);
+
 /* Device-side status of the last ssd_fwd that used `workspace` on `stream`:
  * synchronises `stream`, then returns SSD_OK, SSD_ERR_TIMEOUT or
  * SSD_ERR_BAD_SEQLENS (or SSD_ERR_CUDA if the copy fails). */

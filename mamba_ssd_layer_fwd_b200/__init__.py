@@ -22,7 +22,7 @@ import threading
 from typing import Optional
 
 __all__ = [
-    "ssd_fwd", "SsdParams", "workspace_size", "launch_count", "resolved_path", "library",
+    "ssd_fwd", "ssd_decode_step", "SsdParams", "SsdStepParams", "workspace_size", "launch_count", "resolved_path", "library",
     "library_path", "STATUS", "PATHS", "SsdError",
 ]
 
@@ -36,7 +36,7 @@ STATUS = {0: "SSD_OK", -1: "SSD_ERR_INVALID_ARG", -2: "SSD_ERR_UNSUPPORTED", -3:
 PATHS = {"auto": 0, "simt": 1, "tensor": 2}
 DTYPES = {"f32": 0, "bf16": 1}
 
-EXPORTED = ("ssd_fwd", "ssd_fwd_workspace_size", "ssd_get_status", "ssd_fwd_launch_count",
+EXPORTED = ("ssd_fwd", "ssd_decode_step", "ssd_fwd_workspace_size", "ssd_get_status", "ssd_fwd_launch_count",
             "ssd_fwd_resolved_path", "ssd_status_string", "ssd_abi_version")
 
 
@@ -57,6 +57,14 @@ class SsdParams(ctypes.Structure):
     ]
 
 
+class SsdStepParams(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int), ("nheads", ctypes.c_int), ("headdim", ctypes.c_int),
+        ("dstate", ctypes.c_int), ("ngroups", ctypes.c_int), ("io_dtype", ctypes.c_int),
+        ("dt_softplus", ctypes.c_int),
+    ]
+
+
 def library_path() -> str:
     return _LIB_PATH
 
@@ -73,6 +81,8 @@ def library():
             vp, sz, i32, pp = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.POINTER(SsdParams)
             lib.ssd_fwd.restype = i32
             lib.ssd_fwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+            lib.ssd_decode_step.restype = i32
+            lib.ssd_decode_step.argtypes = [ctypes.POINTER(SsdStepParams), vp, vp, vp, vp, vp, vp, vp, vp, vp]
             lib.ssd_fwd_workspace_size.restype = sz
             lib.ssd_fwd_workspace_size.argtypes = [pp]
             lib.ssd_get_status.restype = i32
@@ -204,3 +214,39 @@ def ssd_fwd(x, dt, A_log, B, C, D=None, chunk_len: int = 256, initial_states=Non
         if rc != 0:
             raise SsdError(rc, "ssd_fwd (device status)")
     return (y, final_states) if want_final else y
+
+
+def ssd_decode_step(x, dt, A_log, B, C, D, state, y=None, dt_softplus: bool = True, stream=None):
+    """One decoding step of every row through the C ABI; updates `state` in
+    place and returns y.
+
+    x (batch, nheads, headdim) and dt (batch, nheads), B and C (batch, ngroups,
+    dstate) share the io dtype (bfloat16 or float32); A_log, D (nheads) and
+    state (batch, nheads, headdim, dstate) are float32 on x's device.
+    """
+    import torch
+    lib = library()
+    dev = x.device
+    if dev.type != "cuda":
+        raise ValueError("ssd_decode_step runs on CUDA tensors only")
+    if x.dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError(f"x must be bfloat16 or float32, got {x.dtype}")
+    for name, t in (("x", x), ("dt", dt), ("B", B), ("C", C)):
+        if t.dtype != x.dtype or not t.is_contiguous() or t.device != dev:
+            raise ValueError(f"{name} must be a contiguous {x.dtype} tensor on {dev}")
+    for name, t in (("A_log", A_log), ("D", D), ("state", state)):
+        if t is not None and (t.dtype != torch.float32 or not t.is_contiguous() or t.device != dev):
+            raise ValueError(f"{name} must be a contiguous float32 tensor on {dev}")
+    b, H, P = x.shape
+    G, N = B.shape[1], B.shape[2]
+    if tuple(dt.shape) != (b, H) or tuple(C.shape) != (b, G, N) or tuple(state.shape) != (b, H, P, N):
+        raise ValueError("shape mismatch between x, dt, B, C, state")
+    if y is None:
+        y = torch.empty_like(x)
+    p = SsdStepParams(int(b), int(H), int(P), int(N), int(G), DTYPES["bf16" if x.dtype == torch.bfloat16 else "f32"],
+                      int(bool(dt_softplus)))
+    rc = lib.ssd_decode_step(ctypes.byref(p), _ptr(x), _ptr(dt), _ptr(A_log), _ptr(B), _ptr(C), _ptr(D),
+                             _ptr(state), _ptr(y), _stream_handle(stream))
+    if rc != 0:
+        raise SsdError(rc, "ssd_decode_step")
+    return y

@@ -95,6 +95,11 @@ WORKLOADS = {
     "varlen32k": Workload("varlen32k", 1, 32768, 48, 64, 128, 1, 256, "bf16",
                            num_seqs=16, with_initial_states=True, with_final_states=True,
                            xbc_std=_scaled(128), dt_shift=3.0, a_log_hi=2.7, init_std=0.1),
+    # one decoding step (recurrent mode) of 64 rows of the 2.7B layer shape,
+    # from a carried state; seqlen 1, chunk_len unused by the step
+    "decode_2p7b": Workload("decode_2p7b", 64, 1, 80, 64, 128, 1, 256, "bf16",
+                             with_initial_states=True, with_final_states=True,
+                             xbc_std=_scaled(128), dt_shift=3.0, a_log_hi=2.7, init_std=0.1),
 }
 
 

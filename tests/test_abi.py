@@ -97,3 +97,25 @@ def test_validation_errors(lib):
 def test_status_strings(lib):
     for code in ssd.STATUS:
         assert lib.ssd_status_string(code)
+
+
+def _step(lib, batch=2, nheads=4, headdim=64, dstate=64, ngroups=1, io="bf16", softplus=1, **ptrs):
+    p = ssd.SsdStepParams(batch, nheads, headdim, dstate, ngroups, ssd.DTYPES[io], softplus)
+    a = dict(x=16, dt=16, A_log=16, B=16, C=16, D=None, state=16, y=16)
+    a.update(ptrs)
+    return lib.ssd_decode_step(ctypes.byref(p), a["x"], a["dt"], a["A_log"], a["B"], a["C"], a["D"],
+                               a["state"], a["y"], None)
+
+
+def test_decode_step_validation(lib):
+    # every call is rejected on the host before anything is launched
+    assert _step(lib, nheads=6, ngroups=4) == -1                 # H % G
+    assert _step(lib, dstate=0) == -1
+    assert _step(lib, softplus=2) == -1
+    assert _step(lib, dstate=30) == -2                           # not a multiple of 4
+    assert _step(lib, dstate=260) == -2                          # above 256
+    assert _step(lib, B=None) == -1
+    assert _step(lib, state=None) == -1
+    assert _step(lib, B=24) == -1                                # misaligned vector operand
+    assert _step(lib, state=8) == -1
+    assert _step(lib, batch=0, x=None, B=None) == 0              # nothing to do
