@@ -55,7 +55,7 @@ constexpr int kThreadsTc = 512;  // 16 warps
 constexpr int kMaskWarps = 6;    // warps 4-7, 10, 11
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kCsd = 4;          // depth of the per-(block, head) cumsum ring
-constexpr int kPrefetch = 3;     // blocks of L2 prefetch ahead of the TMA loads
+constexpr int kPrefetch = 1;     // blocks of L2 prefetch ahead of the TMA loads
 
 struct TcItem {
     int seq;     // sequence index
