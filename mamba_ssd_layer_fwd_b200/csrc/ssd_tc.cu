@@ -151,10 +151,8 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
     // shared array itself, so every access below stays a shared-memory access
     const uint32_t smem_pad = ((smem_u32(smem_raw) + 1023u) & ~1023u) - smem_u32(smem_raw);
     TcSmem<NST> &S = *reinterpret_cast<TcSmem<NST> *>(smem_raw + smem_pad);
-    // dstate 256 keeps more live registers: there the out-of-line wait call spills,
-    // and the UMMA issue loops run faster unrolled
+    // dstate 256 keeps more live registers: there the out-of-line wait call spills
     constexpr bool kInlW = NST >= 256;
-    constexpr int kMmaUnroll = NST >= 256 ? 16 : 1;
     const int item_idx = blockIdx.x;
     if (item_idx >= *prm.count) return;
     const TcItem it = prm.items[item_idx];
@@ -295,7 +293,9 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
     } else if (warp == 1) {
         // ---------------------------------------------- UMMA issuer: state path
         // H_j <- H_j + B_c^T (w o X)   (H_j already rescaled by exp(cs_last) by the state warps)
-        if (lane == 0) {
+        {
+            // the whole warp runs the loop; one elected lane issues
+            const bool leader = elect_one();
             const uint32_t id_h = idesc_bf16_f32(128, kP, true, true);
             const uint32_t id_h2 = idesc_bf16_f32(128, 2 * kP, true, true);
             const uint32_t lbo_m = NST >= 128 ? 16384u : 0u;   // N = 64: rows 64..127 repeat rows 0..63
@@ -314,41 +314,41 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                     SSD_TRACE_EV(15, c * KH);
                     if (!ok) break;
                     tc_fence_after();
-                    const uint32_t sW = smem_u32(S.xw[0]);
-#pragma unroll kMmaUnroll
+                    const uint64_t a0 = sdesc_sw128(sB, lbo_m, 1024), b0 = sdesc_sw128(smem_u32(S.xw[0]), 16384, 1024);
+#pragma unroll
                     for (int kk = 0; kk < kQ / 16; ++kk)
-                        umma_ss(tb + kColH, sdesc_sw128(sB + kk * 2048, lbo_m, 1024),
-                                sdesc_sw128(sW + kk * 2048, 16384, 1024), id_h2, 1);
+                        if (leader) umma_ss(tb + kColH, desc_adv(a0, kk * 2048), desc_adv(b0, kk * 2048), id_h2, 1);
 #pragma unroll
                     for (int j = 0; j < 2; ++j) {
-                        umma_commit(kTmaY ? &S.xw_free[j] : &S.xw_empty[j]);
-                        umma_commit(&S.h_ready[j]);
+                        if (leader) umma_commit(kTmaY ? &S.xw_free[j] : &S.xw_empty[j]);
+                        if (leader) umma_commit(&S.h_ready[j]);
                     }
                     SSD_TRACE_EV(4, c * KH);
-                    umma_commit(&S.bc_empty[bs]);
-                    continue;
-                }
-                for (int j = 0; j < KH && ok; ++j) {
-                    const int u = c * KH + j, wi = u % kXwD;
-                    ok = mbar_wait<kInlW>(&S.xw_full[wi], (u / kXwD) & 1, abort) && mbar_wait<kInlW>(&S.hs_full[j], c & 1, abort);
-                    SSD_TRACE_EV(15, u);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint32_t sW = smem_u32(S.xw[wi]);
+                } else {
+                    for (int j = 0; j < KH && ok; ++j) {
+                        const int u = c * KH + j, wi = u % kXwD;
+                        ok = mbar_wait<kInlW>(&S.xw_full[wi], (u / kXwD) & 1, abort) && mbar_wait<kInlW>(&S.hs_full[j], c & 1, abort);
+                        SSD_TRACE_EV(15, u);
+                        if (!ok) break;
+                        tc_fence_after();
+                        const uint64_t b0 = sdesc_sw128(smem_u32(S.xw[wi]), 16384, 1024);
 #pragma unroll
-                    for (int mt = 0; mt < kMT; ++mt)
-#pragma unroll kMmaUnroll
-                        for (int kk = 0; kk < kQ / 16; ++kk)
-                            umma_ss(tb + kColH + 64 * (j * kMT + mt),
-                                    sdesc_sw128(sB + mt * 32768 + kk * 2048, lbo_m, 1024),
-                                    sdesc_sw128(sW + kk * 2048, 16384, 1024), id_h, 1);
-                    umma_commit(kTmaY ? &S.xw_free[wi] : &S.xw_empty[wi]);
-                    umma_commit(&S.h_ready[j]);
-                    SSD_TRACE_EV(4, u);
+                        for (int mt = 0; mt < kMT; ++mt) {
+                            const uint64_t a0 = sdesc_sw128(sB + mt * 32768, lbo_m, 1024);
+#pragma unroll
+                            for (int kk = 0; kk < kQ / 16; ++kk)
+                                if (leader)
+                                    umma_ss(tb + kColH + 64 * (j * kMT + mt), desc_adv(a0, kk * 2048),
+                                            desc_adv(b0, kk * 2048), id_h, 1);
+                        }
+                        if (leader) umma_commit(kTmaY ? &S.xw_free[wi] : &S.xw_empty[wi]);
+                        if (leader) umma_commit(&S.h_ready[j]);
+                        SSD_TRACE_EV(4, u);
+                    }
                 }
-                umma_commit(&S.bc_empty[bs]);
+                if (leader) umma_commit(&S.bc_empty[bs]);
             }
-            umma_commit(&S.drain_s);
+            if (leader) umma_commit(&S.drain_s);
             mbar_wait<kInlW>(&S.drain_s, 0, abort, 200000000ull);
         }
     } else if (warp == 2) {
@@ -406,7 +406,9 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
         }
     } else if (warp == 3) {
         // --------------------------------------------- UMMA issuer: output path
-        if (!STATE_ONLY && lane == 0) {
+        if (!STATE_ONLY) {
+            // the whole warp runs the loop; one elected lane issues
+            const bool leader = elect_one();
             const uint32_t id_cb = idesc_bf16_f32(128, 128, false, false);
             const uint32_t id_y = idesc_bf16_f32(128, kP, false, true);
             bool ok = true;
@@ -416,15 +418,14 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                 if (!mbar_wait<kInlW>(&S.bc_full[bs], (c / kSt) & 1, abort)) return false;
                 if (c >= 1 && !mbar_wait<kInlW>(&S.cb_empty, (c - 1) & 1, abort)) return false;
                 tc_fence_after();
-                const uint32_t sC = smem_u32(S.bc[bs][0][0]);
-                const uint32_t sB = smem_u32(S.bc[bs][1][0]);
-#pragma unroll kMmaUnroll
+                const uint64_t a0 = sdesc_sw128(smem_u32(S.bc[bs][0][0]), 16, 1024);
+                const uint64_t b0 = sdesc_sw128(smem_u32(S.bc[bs][1][0]), 16, 1024);
+#pragma unroll
                 for (int kk = 0; kk < NST / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    umma_ss(tb + kColCB, sdesc_sw128(sC + off, 16, 1024), sdesc_sw128(sB + off, 16, 1024), id_cb,
-                            kk > 0);
+                    if (leader) umma_ss(tb + kColCB, desc_adv(a0, off), desc_adv(b0, off), id_cb, kk > 0);
                 }
-                umma_commit(&S.cb_full);
+                if (leader) umma_commit(&S.cb_full);
                 SSD_TRACE_EV(2, c);
                 return true;
             };
@@ -447,14 +448,13 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                     SSD_TRACE_EV(17, u);
                     if (!ok) break;
                     tc_fence_after();
-                    const uint32_t sH = smem_u32(S.hbf);
-#pragma unroll kMmaUnroll
+                    const uint64_t a0 = sdesc_sw128(sC, 16, 1024), b0 = sdesc_sw128(smem_u32(S.hbf), 16384, 1024);
+#pragma unroll
                     for (int kk = 0; kk < NST / 16; ++kk) {
                         const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                        umma_ss(tb + kColYo, sdesc_sw128(sC + off, 16, 1024),
-                                sdesc_sw128(sH + kk * 2048, 16384, 1024), id_y, kk > 0);
+                        if (leader) umma_ss(tb + kColYo, desc_adv(a0, off), desc_adv(b0, kk * 2048), id_y, kk > 0);
                     }
-                    umma_commit(&S.hb_empty);
+                    if (leader) umma_commit(&S.hb_empty);
                     SSD_TRACE_EV(3, u);
                     // the next block's CB runs while the mask warps finish this block's last head
                     if (kSt > 1 && j == KH - 1 && c + 1 < nblk) {
@@ -468,20 +468,20 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                     SSD_TRACE_EV(16, u);
                     if (!ok) break;
                     tc_fence_after();
-                    const uint32_t sX = smem_u32(S.x[xs]);
-#pragma unroll kMmaUnroll
+                    const uint64_t x0 = sdesc_sw128(smem_u32(S.x[xs]), 16384, 1024);
+                    const uint32_t pm = tb + kColPm + 64 * pi;
+#pragma unroll
                     for (int kk = 0; kk < kQ / 16; ++kk)
-                        umma_ts(tb + kColYd, tb + kColPm + 64 * pi + kk * 8,
-                                sdesc_sw128(sX + kk * 2048, 16384, 1024), id_y, kk > 0);
-                    umma_commit(&S.pm_empty[pi]);
-                    umma_commit(&S.y_full);
-                    umma_commit(&S.x_empty[xs]);
+                        if (leader) umma_ts(tb + kColYd, pm + kk * 8, desc_adv(x0, kk * 2048), id_y, kk > 0);
+                    if (leader) umma_commit(&S.pm_empty[pi]);
+                    if (leader) umma_commit(&S.y_full);
+                    if (leader) umma_commit(&S.x_empty[xs]);
                     SSD_TRACE_EV(5, u);
                 }
-                umma_commit(&S.bc_empty[bs]);
+                if (leader) umma_commit(&S.bc_empty[bs]);
             }
             // every UMMA issued so far has completed before TMEM is released
-            umma_commit(&S.drain_o);
+            if (leader) umma_commit(&S.drain_o);
             mbar_wait<kInlW>(&S.drain_o, 0, abort, 200000000ull);
         }
     } else if ((warp >= 4 && warp < 8) || warp == 10 || warp == 11) {

@@ -145,6 +145,20 @@ __device__ __forceinline__ void fence_async_smem()
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// One lane of the (converged) warp, chosen by the hardware: the lane that
+// issues single-thread instructions (UMMA, commit) while the whole warp runs
+// the control flow and keeps the operand descriptors warp-uniform.
+__device__ __forceinline__ bool elect_one()
+{
+    uint32_t leader = 0;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t"
+        "elect.sync _|P, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, P;\n\t}"
+        : "=r"(leader));
+    return leader != 0;
+}
+
 // ------------------------------------------------------------------ tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t *dst, uint32_t ncols)   // whole warp
 {
@@ -244,6 +258,15 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
 {
     return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
            ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// The descriptor of the same operand `bytes` further on: the start-address
+// field is the low 14 bits (address >> 4) and shared addresses stay below
+// 256 KB, so the add never carries out of it.  One add per UMMA keeps the
+// issuing thread's dependency chain short.
+__device__ __forceinline__ uint64_t desc_adv(uint64_t desc, uint32_t bytes)
+{
+    return desc + (uint64_t)(bytes >> 4);
 }
 
 // Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulator.
