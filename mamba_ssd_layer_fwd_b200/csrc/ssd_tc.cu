@@ -544,35 +544,44 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                                 __syncwarp();
                                 if (lane == 0) mbar_arrive(&S.cb_empty);
                             }
+                            float m[32];
                             if (!exact) {
-                                // exp2(cs2_l - cs2_s) delta_s = exp2(cs2_l - R) * exp2(R - cs2_s) delta_s
+                                // exp2(cs2_l - cs2_s) delta_s = exp2(cs2_l - R) * [exp2(R - cs2_s) delta_s]:
+                                // CB times the column factor, then the row factor of each 16-column chunk
                                 const float v0 = ex2_approx(rowc - R0), v1 = ex2_approx(rowc - R1);
 #pragma unroll
-                                for (int i = 0; i < 32; ++i) cf[i] *= (i < 16 ? v0 : v1);
+                                for (int i = 0; i < 32; i += 2)
+                                    mul_f32x2(m[i], m[i + 1], __uint_as_float(r[i]), __uint_as_float(r[i + 1]), cf[i],
+                                              cf[i + 1]);
+#pragma unroll
+                                for (int i = 0; i < 32; i += 2) {
+                                    const float v = i < 16 ? v0 : v1;
+                                    mul_f32x2(m[i], m[i + 1], m[i], m[i + 1], v, v);
+                                }
                             } else {
                                 const float4 *cc = reinterpret_cast<const float4 *>(&S.cs2[slot][s0]);
                                 const float4 *dd = reinterpret_cast<const float4 *>(&S.dl[slot][s0]);
 #pragma unroll
                                 for (int i4 = 0; i4 < 8; ++i4) {
                                     const float4 c4 = cc[i4], d4 = dd[i4];
-                                    cf[4 * i4 + 0] = ex2_approx(rowc - c4.x) * d4.x;
-                                    cf[4 * i4 + 1] = ex2_approx(rowc - c4.y) * d4.y;
-                                    cf[4 * i4 + 2] = ex2_approx(rowc - c4.z) * d4.z;
-                                    cf[4 * i4 + 3] = ex2_approx(rowc - c4.w) * d4.w;
+                                    m[4 * i4 + 0] = __uint_as_float(r[4 * i4 + 0]) * (ex2_approx(rowc - c4.x) * d4.x);
+                                    m[4 * i4 + 1] = __uint_as_float(r[4 * i4 + 1]) * (ex2_approx(rowc - c4.y) * d4.y);
+                                    m[4 * i4 + 2] = __uint_as_float(r[4 * i4 + 2]) * (ex2_approx(rowc - c4.z) * d4.z);
+                                    m[4 * i4 + 3] = __uint_as_float(r[4 * i4 + 3]) * (ex2_approx(rowc - c4.w) * d4.w);
+                                }
+                            }
+                            // pairs are 32-aligned like the warp's rows: only the pair holding the
+                            // warp's diagonal block needs the causal edge (s > l is zero, s == l gains D)
+                            if (s0 + 31 >= q * 32) {            // warp-uniform
+#pragma unroll
+                                for (int i = 0; i < 32; ++i) {
+                                    const int sa = s0 + i;
+                                    m[i] = sa < l ? m[i] : (sa == l ? m[i] + Dh : 0.0f);
                                 }
                             }
                             uint32_t packed[16];
 #pragma unroll
-                            for (int i2 = 0; i2 < 16; ++i2) {
-                                const int sa = s0 + 2 * i2;
-                                float ma = __uint_as_float(r[2 * i2]) * cf[2 * i2];
-                                float mb = __uint_as_float(r[2 * i2 + 1]) * cf[2 * i2 + 1];
-                                if (sa + 1 >= l) {              // causal edge: s > l is zero, s == l gains D
-                                    ma = sa < l ? ma : (sa == l ? ma + Dh : 0.0f);
-                                    mb = sa + 1 < l ? mb : (sa + 1 == l ? mb + Dh : 0.0f);
-                                }
-                                packed[i2] = pack_bf16x2(ma, mb);
-                            }
+                            for (int i2 = 0; i2 < 16; ++i2) packed[i2] = pack_bf16x2(m[2 * i2], m[2 * i2 + 1]);
                             tmem_st16(pm_col + pair * 16, packed);
                         } else {                                // above the diagonal for every row
                             uint32_t zeros[16];
@@ -734,8 +743,10 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
                             const int pp = q8 + 2 * i;
-                            pk[i] = pack_bf16x2(__uint_as_float(yd[pp]) + el * __uint_as_float(yo[h0 + pp]),
-                                                __uint_as_float(yd[pp + 1]) + el * __uint_as_float(yo[h0 + pp + 1]));
+                            float ya, yb;
+                            fma_f32x2(ya, yb, el, el, __uint_as_float(yo[h0 + pp]), __uint_as_float(yo[h0 + pp + 1]),
+                                      __uint_as_float(yd[pp]), __uint_as_float(yd[pp + 1]));
+                            pk[i] = pack_bf16x2(ya, yb);
                         }
                         const uint4 v4 = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                         if (via_tma)
@@ -800,7 +811,12 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                             make_uint4(pk[4], pk[5], pk[6], pk[7]);
                     }
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) r[p0 + i] = __float_as_uint(alpha * __uint_as_float(r[p0 + i]));
+                    for (int i = 0; i < 16; i += 2) {
+                        float ha, hb;
+                        mul_f32x2(ha, hb, alpha, alpha, __uint_as_float(r[p0 + i]), __uint_as_float(r[p0 + i + 1]));
+                        r[p0 + i] = __float_as_uint(ha);
+                        r[p0 + i + 1] = __float_as_uint(hb);
+                    }
                     tmem_st16(hcol + p0, *reinterpret_cast<uint32_t(*)[16]>(&r[p0]));
                 }
             }

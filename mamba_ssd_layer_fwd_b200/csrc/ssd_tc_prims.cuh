@@ -286,6 +286,33 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t col)
     return row * 128u + ((((col >> 3) ^ (row & 7u)) & 7u) << 4) + ((col & 7u) << 1);
 }
 
+// Two fp32 products in one instruction (sm_100 paired fp32 pipe, round to
+// nearest): (d0, d1) = (a0 * b0, a1 * b1).
+__device__ __forceinline__ void mul_f32x2(float &d0, float &d1, float a0, float a1, float b0, float b1)
+{
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// (d0, d1) = (a0 * b0 + c0, a1 * b1 + c1), each a single-rounding fused multiply-add.
+__device__ __forceinline__ void fma_f32x2(float &d0, float &d1, float a0, float a1, float b0, float b1, float c0,
+                                          float c1)
+{
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "mov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
 // 2^x with the hardware approximation (MUFU.EX2); flushes denormals. Used
 // where the result is rounded to bf16 right after.
 __device__ __forceinline__ float ex2_approx(float x)
