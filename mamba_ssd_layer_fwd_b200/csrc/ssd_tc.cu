@@ -172,8 +172,6 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
     // two w o X slots, so the next unit's w o X pass runs meanwhile.
     constexpr bool kTmaY = !STATE_ONLY && kXwD >= 2;
     constexpr int kMT = NST >= 256 ? 2 : 1;        // 128-row state tiles per head (H^T rows = n)
-    // two heads whose w o X tiles fill the two-slot ring: one state UMMA per block
-    constexpr bool kMergeH = KH == 2 && kXwD == 2 && kMT == 1;
 
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
@@ -297,7 +295,6 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             // the whole warp runs the loop; one elected lane issues
             const bool leader = elect_one();
             const uint32_t id_h = idesc_bf16_f32(128, kP, true, true);
-            const uint32_t id_h2 = idesc_bf16_f32(128, 2 * kP, true, true);
             const uint32_t lbo_m = NST >= 128 ? 16384u : 0u;   // N = 64: rows 64..127 repeat rows 0..63
             bool ok = true;
             for (int c = 0; c < nblk && ok; ++c) {
@@ -305,46 +302,25 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                 ok = mbar_wait<kInlW>(&S.bc_full[bs], (c / kSt) & 1, abort);
                 if (!ok) break;
                 const uint32_t sB = smem_u32(S.bc[bs][1][0]);
-                if (kMergeH) {
-                    // both heads in one N = 128 UMMA: their w o X tiles sit in adjacent slots
-                    // (the 16 KB slot stride is the descriptor's stride between 64-column
-                    // blocks) and their states in adjacent TMEM columns, so B^T is read once
-                    ok = mbar_wait<kInlW>(&S.xw_full[0], c & 1, abort) && mbar_wait<kInlW>(&S.xw_full[1], c & 1, abort) &&
-                         mbar_wait<kInlW>(&S.hs_full[0], c & 1, abort) && mbar_wait<kInlW>(&S.hs_full[1], c & 1, abort);
-                    SSD_TRACE_EV(15, c * KH);
+                for (int j = 0; j < KH && ok; ++j) {
+                    const int u = c * KH + j, wi = u % kXwD;
+                    ok = mbar_wait<kInlW>(&S.xw_full[wi], (u / kXwD) & 1, abort) && mbar_wait<kInlW>(&S.hs_full[j], c & 1, abort);
+                    SSD_TRACE_EV(15, u);
                     if (!ok) break;
                     tc_fence_after();
-                    const uint64_t a0 = sdesc_sw128(sB, lbo_m, 1024), b0 = sdesc_sw128(smem_u32(S.xw[0]), 16384, 1024);
+                    const uint64_t b0 = sdesc_sw128(smem_u32(S.xw[wi]), 16384, 1024);
 #pragma unroll
-                    for (int kk = 0; kk < kQ / 16; ++kk)
-                        if (leader) umma_ss(tb + kColH, desc_adv(a0, kk * 2048), desc_adv(b0, kk * 2048), id_h2, 1);
+                    for (int mt = 0; mt < kMT; ++mt) {
+                        const uint64_t a0 = sdesc_sw128(sB + mt * 32768, lbo_m, 1024);
 #pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        if (leader) umma_commit(kTmaY ? &S.xw_free[j] : &S.xw_empty[j]);
-                        if (leader) umma_commit(&S.h_ready[j]);
+                        for (int kk = 0; kk < kQ / 16; ++kk)
+                            if (leader)
+                                umma_ss(tb + kColH + 64 * (j * kMT + mt), desc_adv(a0, kk * 2048),
+                                        desc_adv(b0, kk * 2048), id_h, 1);
                     }
-                    SSD_TRACE_EV(4, c * KH);
-                } else {
-                    for (int j = 0; j < KH && ok; ++j) {
-                        const int u = c * KH + j, wi = u % kXwD;
-                        ok = mbar_wait<kInlW>(&S.xw_full[wi], (u / kXwD) & 1, abort) && mbar_wait<kInlW>(&S.hs_full[j], c & 1, abort);
-                        SSD_TRACE_EV(15, u);
-                        if (!ok) break;
-                        tc_fence_after();
-                        const uint64_t b0 = sdesc_sw128(smem_u32(S.xw[wi]), 16384, 1024);
-#pragma unroll
-                        for (int mt = 0; mt < kMT; ++mt) {
-                            const uint64_t a0 = sdesc_sw128(sB + mt * 32768, lbo_m, 1024);
-#pragma unroll
-                            for (int kk = 0; kk < kQ / 16; ++kk)
-                                if (leader)
-                                    umma_ss(tb + kColH + 64 * (j * kMT + mt), desc_adv(a0, kk * 2048),
-                                            desc_adv(b0, kk * 2048), id_h, 1);
-                        }
-                        if (leader) umma_commit(kTmaY ? &S.xw_free[wi] : &S.xw_empty[wi]);
-                        if (leader) umma_commit(&S.h_ready[j]);
-                        SSD_TRACE_EV(4, u);
-                    }
+                    if (leader) umma_commit(kTmaY ? &S.xw_free[wi] : &S.xw_empty[wi]);
+                    if (leader) umma_commit(&S.h_ready[j]);
+                    SSD_TRACE_EV(4, u);
                 }
                 if (leader) umma_commit(&S.bc_empty[bs]);
             }
