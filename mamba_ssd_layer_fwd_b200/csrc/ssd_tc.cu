@@ -861,14 +861,19 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
 }
 
 // ---------------------------------------------------------------- planning
-// Work items: (sequence, head block, segment).  One block of 1024 threads.
+// Work items: (sequence, head block, segment), item index = global segment *
+// n_hb + head block.  One block of 1024 threads: per chunk of 1024 sequences a
+// block-wide scan places each sequence's segments, then every thread writes
+// items (one per (segment, head block)); seqseg[s] = first global segment of a
+// sequence cut into two or more segments (-1 otherwise) for the segment scan.
 __global__ void __launch_bounds__(1024)
 tc_plan_kernel(const int32_t *__restrict__ cu_seqlens, int nseq, int seqlen, int seg_len, int n_hb, int KH,
                TcItem *items, int *count, int max_items, int *status, const float *__restrict__ init,
-               float *__restrict__ final_states, int H, int PN)
+               float *__restrict__ final_states, int H, int PN, int *seqseg)
 {
     __shared__ int s_bad, s_carry;
     __shared__ int s_warp[32];
+    __shared__ int s_incl[1024], s_tok0[1024], s_len[1024];
     const int tid = threadIdx.x;
     if (tid == 0) {
         *status = 0;
@@ -892,6 +897,7 @@ tc_plan_kernel(const int32_t *__restrict__ cu_seqlens, int nseq, int seqlen, int
     }
     for (int base = 0; base < nseq; base += 1024) {
         const int i = base + tid;
+        const int cnt = min(1024, nseq - base);
         int tok0 = 0, len = 0, ns = 0;
         if (i < nseq) {
             tok0 = cu_seqlens ? cu_seqlens[i] : i * seqlen;
@@ -914,59 +920,65 @@ tc_plan_kernel(const int32_t *__restrict__ cu_seqlens, int nseq, int seqlen, int
             s_warp[tid] = w;
         }
         __syncthreads();
-        const int incl = v + ((tid >> 5) ? s_warp[(tid >> 5) - 1] : 0) + s_carry;
-        const int gseg0 = incl - ns;
-        if (i < nseq) {
-            for (int sg = 0; sg < ns; ++sg) {
-                const int gs = gseg0 + sg;
-                for (int hb = 0; hb < n_hb; ++hb) {
-                    const int idx = gs * n_hb + hb;
-                    if (idx < max_items) {
-                        TcItem t;
-                        t.seq = i;
-                        t.tok0 = tok0 + sg * seg_len;
-                        t.len = min(seg_len, len - sg * seg_len);
-                        t.gseg = gs;
-                        t.seg = sg;
-                        t.nseg = ns;
-                        t.h0 = hb * KH;
-                        t.pad = 0;
-                        items[idx] = t;
-                    }
-                }
+        const int incl = v + ((tid >> 5) ? s_warp[(tid >> 5) - 1] : 0);   // segments up to i, in this chunk
+        const int carry = s_carry;
+        s_incl[tid] = incl;
+        s_tok0[tid] = tok0;
+        s_len[tid] = len;
+        if (i < nseq && seqseg) seqseg[i] = ns >= 2 ? carry + incl - ns : -1;
+        __syncthreads();
+        const int chunk_segs = s_incl[cnt - 1];
+        for (int idx = tid; idx < chunk_segs * n_hb; idx += 1024) {
+            const int sl = idx / n_hb, hb = idx - sl * n_hb;
+            // the sequence holding chunk segment sl: first k with incl[k] > sl
+            int lo = 0, hi = cnt - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (s_incl[mid] > sl) hi = mid; else lo = mid + 1;
+            }
+            const int first = lo ? s_incl[lo - 1] : 0;   // chunk segment where sequence lo starts
+            const int segi = sl - first;
+            const int gs = carry + sl;
+            const int item = gs * n_hb + hb;
+            if (item < max_items) {
+                TcItem t;
+                t.seq = base + lo;
+                t.tok0 = s_tok0[lo] + segi * seg_len;
+                t.len = min(seg_len, s_len[lo] - segi * seg_len);
+                t.gseg = gs;
+                t.seg = segi;
+                t.nseg = s_incl[lo] - first;
+                t.h0 = hb * KH;
+                t.pad = 0;
+                items[item] = t;
+            }
+        }
+        // empty sequences: the final state is the initial state
+        if (final_states) {
+            for (int k2 = 0; k2 < cnt; ++k2) {
+                if (s_len[k2] != 0) continue;
+                const size_t o = (size_t)(base + k2) * H * PN;
+                for (int e = tid; e < H * PN; e += 1024) final_states[o + e] = init ? init[o + e] : 0.0f;
             }
         }
         __syncthreads();
-        if (tid == 1023) s_carry = incl;
+        if (tid == 0) s_carry = carry + chunk_segs;
         __syncthreads();
     }
     if (tid == 0) *count = min(s_carry * n_hb, max_items);
-    // empty sequences: the final state is the initial state
-    if (final_states) {
-        for (int i = 0; i < nseq; ++i) {
-            const int len = cu_seqlens ? cu_seqlens[i + 1] - cu_seqlens[i] : seqlen;
-            if (len != 0) continue;
-            for (int e = tid; e < H * PN; e += 1024)
-                final_states[(size_t)i * H * PN + e] = init ? init[(size_t)i * H * PN + e] : 0.0f;
-        }
-    }
 }
 
 // Segment scan: entering state of every segment of every sequence,
 // H_in(0) = initial state, H_in(k+1) = exp(ldec_k) H_in(k) + S_k; written in
 // place over the pass-1 end states.
 __global__ void __launch_bounds__(256)
-tc_seg_scan_kernel(const TcItem *__restrict__ items, const int *__restrict__ count, int n_hb, int nseq_items_stride,
-                   float *segstate, const float *__restrict__ seglogdec, const float *__restrict__ init, int H,
-                   int PN)
+tc_seg_scan_kernel(const TcItem *__restrict__ items, const int *__restrict__ seqseg, int n_hb, float *segstate,
+                   const float *__restrict__ seglogdec, const float *__restrict__ init, int H, int PN)
 {
-    (void)nseq_items_stride;
-    // grid: (first-segment items / n_hb, H, ceil(PN / 256)); blockIdx.x indexes global segments
-    const int gs = blockIdx.x;
-    const int cnt = *count / n_hb;
-    if (gs >= cnt) return;
+    // grid: (sequences, H, ceil(PN / 256)); only sequences cut into two or more segments work
+    const int gs = seqseg[blockIdx.x];
+    if (gs < 0) return;
     const TcItem it = items[(size_t)gs * n_hb];
-    if (it.seg != 0 || it.nseg < 2) return;   // one thread group per multi-segment sequence
     const int h = blockIdx.y;
     const int e = blockIdx.z * 256 + threadIdx.x;
     if (e >= PN) return;
@@ -1132,6 +1144,8 @@ size_t tc_workspace_bytes(const ssd_fwd_params &p)
     if (s.segmented) {
         b += align256((size_t)s.max_segments * p.nheads * kP * p.dstate * sizeof(float));
         b += align256((size_t)s.max_segments * p.nheads * sizeof(float));
+        const int nseq = p.num_seqs > 0 ? p.num_seqs : p.batch;
+        b += align256((size_t)nseq * sizeof(int));
     }
     return b;
 }
@@ -1146,17 +1160,20 @@ cudaError_t launch_tc(const ssd_fwd_params &p, const Plan &plan, const Dims &d, 
     TcItem *items = reinterpret_cast<TcItem *>(ws);
     size_t off = align256(sizeof(TcItem) * (size_t)s.max_items);
     float *segstate = nullptr, *seglogdec = nullptr;
+    int *seqseg = nullptr;
     if (s.segmented) {
         segstate = reinterpret_cast<float *>(ws + off);
         off += align256((size_t)s.max_segments * p.nheads * kP * p.dstate * sizeof(float));
         seglogdec = reinterpret_cast<float *>(ws + off);
+        off += align256((size_t)s.max_segments * p.nheads * sizeof(float));
+        seqseg = reinterpret_cast<int *>(ws + off);
     }
     const long long tokens = (long long)p.batch * p.seqlen;
     const int PN = kP * p.dstate;
     const int nseq = plan.nseq;
     tc_plan_kernel<<<1, 1024, 0, stream>>>(a.cu_seqlens, nseq, p.seqlen, s.seg_len, s.n_hb, s.KH, items,
                                            plan.count, s.max_items, plan.status, a.init, a.final_states,
-                                           p.nheads, PN);
+                                           p.nheads, PN, seqseg);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || tokens == 0) return e;
 
@@ -1190,9 +1207,8 @@ cudaError_t launch_tc(const ssd_fwd_params &p, const Plan &plan, const Dims &d, 
     if (s.segmented) {
         e = launch_walk_any<true>(p.dstate, s.KH, s.max_items, mX, mB, mC, mY, prm, stream);
         if (e != cudaSuccess) return e;
-        const dim3 gs(s.max_segments, p.nheads, (PN + 255) / 256);
-        tc_seg_scan_kernel<<<gs, 256, 0, stream>>>(items, plan.count, s.n_hb, 0, segstate, seglogdec, a.init,
-                                                   p.nheads, PN);
+        const dim3 gs(nseq, p.nheads, (PN + 255) / 256);
+        tc_seg_scan_kernel<<<gs, 256, 0, stream>>>(items, seqseg, s.n_hb, segstate, seglogdec, a.init, p.nheads, PN);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (prof_begin) cudaEventRecord(prof_begin, stream);
