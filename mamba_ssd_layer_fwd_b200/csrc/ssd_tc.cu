@@ -75,9 +75,12 @@ struct TcParams {
     float *final_states;
     float *segstate;      // [max_segments][H][P][N]: pass-1 end states, then entering states
     float *seglogdec;     // [max_segments][H]: sum of delta*A over the segment
-    const TcItem *items;
+    const TcItem *items;  // null: equal-length rows of one segment each (see direct_base)
     const int *count;
     int *status;
+    // items == null: item i of this launch covers heads row * H + h0 .. + KH - 1 of
+    // the flattened (row, head) index g = direct_base + i * KH; n_items items
+    int n_items, direct_base, seqlen;
     int H, G, N, heads_per_group;
     int dt_softplus;
     int withhold_x0;      // testing: work item 0 never loads its first x tile (bounded waits expire)
@@ -164,8 +167,23 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
     // dstate 256 keeps more live registers: there the out-of-line wait call spills
     constexpr bool kInlW = NST >= 256;
     const int item_idx = blockIdx.x;
-    if (item_idx >= *prm.count) return;
-    const TcItem it = prm.items[item_idx];
+    TcItem it;
+    if (prm.items) {
+        if (item_idx >= *prm.count) return;
+        it = prm.items[item_idx];
+    } else {
+        if (item_idx >= prm.n_items) return;
+        const int g0 = prm.direct_base + item_idx * KH;
+        const int row = g0 / prm.H;
+        it.seq = row;
+        it.tok0 = row * prm.seqlen;
+        it.len = prm.seqlen;
+        it.gseg = row;
+        it.seg = 0;
+        it.nseg = 1;
+        it.h0 = g0 - row * prm.H;
+        it.pad = 0;
+    }
     if (STATE_ONLY && it.seg >= it.nseg - 1) return;   // only non-final segments need end states
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1150,7 +1168,32 @@ size_t tc_workspace_bytes(const ssd_fwd_params &p)
     return b;
 }
 
-int tc_launch_count(const ssd_fwd_params &p) { return plan_shape(p).segmented ? 4 : 2; }
+// Equal-length rows that need no segmentation: every work item is (row, head
+// block) and the walk derives it from its block index, so no planner runs.
+bool direct_items(const ssd_fwd_params &p, const TcPlanShape &s)
+{
+    return p.num_seqs == 0 && !s.segmented && (long long)p.batch * p.seqlen > 0;
+}
+
+// Direct items with two heads each that do not fill whole waves of the SMs:
+// the first whole waves run as two-head items, the pairs left over as twice as
+// many one-head items in a second launch, which take about half as long (a
+// last round of a few two-head items would leave most SMs idle for a whole
+// item).  Returns the number of two-head items of the first launch, or -1
+// for a single launch.
+int direct_split(const ssd_fwd_params &p, const TcPlanShape &s)
+{
+    if (!direct_items(p, s) || s.KH != 2) return -1;
+    const int waves = s.max_items / kPlanSMs;
+    if (waves < 1 || s.max_items % kPlanSMs == 0) return -1;
+    return waves * kPlanSMs;
+}
+
+int tc_launch_count(const ssd_fwd_params &p)
+{
+    const TcPlanShape s = plan_shape(p);
+    return s.segmented ? 4 : direct_items(p, s) ? (direct_split(p, s) >= 0 ? 2 : 1) : 2;
+}
 
 cudaError_t launch_tc(const ssd_fwd_params &p, const Plan &plan, const Dims &d, const TcArgs &a,
                       cudaStream_t stream, cudaEvent_t prof_begin, cudaEvent_t prof_end)
@@ -1171,10 +1214,17 @@ cudaError_t launch_tc(const ssd_fwd_params &p, const Plan &plan, const Dims &d, 
     const long long tokens = (long long)p.batch * p.seqlen;
     const int PN = kP * p.dstate;
     const int nseq = plan.nseq;
-    tc_plan_kernel<<<1, 1024, 0, stream>>>(a.cu_seqlens, nseq, p.seqlen, s.seg_len, s.n_hb, s.KH, items,
-                                           plan.count, s.max_items, plan.status, a.init, a.final_states,
-                                           p.nheads, PN, seqseg);
-    cudaError_t e = cudaGetLastError();
+    const bool direct = direct_items(p, s);
+    cudaError_t e;
+    if (direct) {
+        // the status word is all the planner would have initialised
+        e = cudaMemsetAsync(plan.status, 0, sizeof(int), stream);
+    } else {
+        tc_plan_kernel<<<1, 1024, 0, stream>>>(a.cu_seqlens, nseq, p.seqlen, s.seg_len, s.n_hb, s.KH, items,
+                                               plan.count, s.max_items, plan.status, a.init, a.final_states,
+                                               p.nheads, PN, seqseg);
+        e = cudaGetLastError();
+    }
     if (e != cudaSuccess || tokens == 0) return e;
 
     CUtensorMap mX, mB, mC, mY;
@@ -1194,8 +1244,11 @@ cudaError_t launch_tc(const ssd_fwd_params &p, const Plan &plan, const Dims &d, 
     prm.final_states = a.final_states;
     prm.segstate = segstate;
     prm.seglogdec = seglogdec;
-    prm.items = items;
+    prm.items = direct ? nullptr : items;
     prm.count = plan.count;
+    prm.n_items = s.max_items;
+    prm.direct_base = 0;
+    prm.seqlen = p.seqlen;
     prm.status = plan.status;
     prm.H = p.nheads;
     prm.G = p.ngroups;
@@ -1212,7 +1265,19 @@ cudaError_t launch_tc(const ssd_fwd_params &p, const Plan &plan, const Dims &d, 
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (prof_begin) cudaEventRecord(prof_begin, stream);
-    e = launch_walk_any<false>(p.dstate, s.KH, s.max_items, mX, mB, mC, mY, prm, stream);
+    const int split = direct_split(p, s);
+    if (split < 0) {
+        e = launch_walk_any<false>(p.dstate, s.KH, s.max_items, mX, mB, mC, mY, prm, stream);
+    } else {
+        prm.n_items = split;
+        e = launch_walk_any<false>(p.dstate, 2, split, mX, mB, mC, mY, prm, stream);
+        if (e == cudaSuccess) {
+            TcParams tail = prm;
+            tail.direct_base = split * 2;
+            tail.n_items = (s.max_items - split) * 2;
+            e = launch_walk_any<false>(p.dstate, 1, tail.n_items, mX, mB, mC, mY, tail, stream);
+        }
+    }
     if (prof_end) cudaEventRecord(prof_end, stream);
     return e;
 }

@@ -107,6 +107,13 @@ def test_single_token_and_empty(path):
     check_full(inp, path=path)
 
 
+def test_tail_items_split_into_single_heads():
+    """160 two-head work items on 148 SMs: the first 148 run as two-head items,
+    the 12 left over as 24 one-head items in a second launch."""
+    inp = small_inputs(batch=2, seqlen=300, H=160, P=64, N=64, G=1, Q=256, init=True, seed=15)
+    check_full(inp, path="tensor")
+
+
 def test_zero_length_batch_passes_initial_state():
     inp = small_inputs(batch=2, seqlen=0, H=2, P=64, N=64, G=1, Q=256, init=True, seed=8)
     y, fin = run_gpu(inp)
