@@ -119,3 +119,30 @@ def test_decode_step_validation(lib):
     assert _step(lib, B=24) == -1                                # misaligned vector operand
     assert _step(lib, state=8) == -1
     assert _step(lib, batch=0, x=None, B=None) == 0              # nothing to do
+
+
+def _tc_params(batch, seqlen, nheads, dstate, ngroups=1, num_seqs=0):
+    return ssd.make_params(batch=batch, seqlen=seqlen, nheads=nheads, headdim=64, dstate=dstate,
+                           ngroups=ngroups, chunk_len=256, num_seqs=num_seqs, io_dtype="bf16", path="auto")
+
+
+def test_tensor_path_work_split(lib):
+    """Host-side work planning of the tensor-core path (no GPU needed): how
+    many kernels one forward launches for each kind of problem."""
+    # 8 x 80 heads: 320 two-head items = 2 whole waves of 148 + 24 pairs run as
+    # 48 one-head items in a second launch; no planner kernel
+    p = _tc_params(8, 2048, 80, 128)
+    assert ssd.resolved_path(p) == "tensor"
+    assert ssd.launch_count(p) == 2
+    # exactly one wave of two-head items: one launch
+    assert ssd.launch_count(_tc_params(148, 256, 2, 64)) == 1
+    # one short row: one item, one launch
+    assert ssd.launch_count(_tc_params(1, 128, 2, 64)) == 1
+    # a 16K-token row with 32 heads: cut into segments (planner, state pass, scan, walk)
+    assert ssd.launch_count(_tc_params(1, 16384, 32, 256, ngroups=8)) == 4
+    # packed variable-length batch: planner + walk, or + state pass + scan when segmented
+    assert ssd.launch_count(_tc_params(1, 32768, 48, 128, num_seqs=16)) == 4
+    assert ssd.launch_count(_tc_params(1, 512, 48, 128, num_seqs=4)) == 2
+    for p in (_tc_params(8, 2048, 80, 128), _tc_params(1, 16384, 32, 256, ngroups=8),
+              _tc_params(1, 32768, 48, 128, num_seqs=16)):
+        assert ssd.workspace_size(p) > 0
