@@ -76,6 +76,14 @@ typedef enum ssd_dtype {
     SSD_DTYPE_BF16 = 1          /* x, dt, B, C, y in bfloat16 (states stay float32) */
 } ssd_dtype;
 
+/* Limits ("see limits" above).  SIMT path: headdim 1..128, dstate 1..256,
+ * float32 or bf16.  Tensor-core path: bf16, headdim 64, dstate 64, 128 or
+ * 256, dt_softplus == 1, chunk_len 128 or 256, at least 128 tokens in the
+ * call; it evaluates the decomposition on 128-token blocks whatever
+ * chunk_len is (the result does not depend on chunk_len beyond rounding).
+ * AUTO takes the tensor-core path whenever these hold.  Requesting a path the
+ * shape does not allow returns SSD_ERR_UNSUPPORTED, and so do problems with
+ * 2^31 or more elements in x or in B, or more than 2^20 packed sequences. */
 typedef enum ssd_path {
     SSD_PATH_AUTO = 0,          /* tensor-core path when the shape allows it, else SIMT */
     SSD_PATH_SIMT = 1,          /* CUDA-core path: any supported shape, float32 or bf16 */
