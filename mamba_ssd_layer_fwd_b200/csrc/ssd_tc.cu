@@ -1062,6 +1062,31 @@ struct TcPlanShape {
 // not depend on which GPU answers), sized for the B200's 148 SMs.
 constexpr int kPlanSMs = 148;
 
+// Segment count (1 = no cut) with the smallest modelled makespan for `rows`
+// equal rows of `nblk` 128-token blocks and `items_per_row` items per row, in
+// block steps of one SM.  Pass 2 runs ceil(items * n / SMs) rounds of items of
+// ceil(blocks / n) blocks; pass 1 (state only, about 0.65 of a pass-2 block)
+// the same over n - 1 segments; each round costs about 1.5 blocks of fill and
+// drain, the segment scan 2.
+long long best_segment_count(long long items, long long nblk)
+{
+    const long long sms = kPlanSMs;
+    long long best_n = 1;
+    double best = 1e300;
+    for (long long n = 1; n <= 64 && n <= nblk; ++n) {
+        const long long bps = (nblk + n - 1) / n;
+        const long long r2 = (items * n + sms - 1) / sms;
+        const long long r1 = n > 1 ? (items * (n - 1) + sms - 1) / sms : 0;
+        const double cost = (double)bps * ((double)r2 + 0.65 * (double)r1) + 1.5 * (double)(r1 + r2) +
+                            (n > 1 ? 2.0 : 0.0);
+        if (cost < best - 1e-9) {
+            best = cost;
+            best_n = n;
+        }
+    }
+    return best_n;
+}
+
 TcPlanShape plan_shape(const ssd_fwd_params &p)
 {
     TcPlanShape s;
@@ -1071,35 +1096,24 @@ TcPlanShape plan_shape(const ssd_fwd_params &p)
     s.n_hb = p.nheads / s.KH;
     const int nseq = p.num_seqs > 0 ? p.num_seqs : p.batch;
     const long long tokens = (long long)p.batch * p.seqlen;
-    const int target = 2 * kPlanSMs;                  // work items wanted (two per SM)
+    const long long items = (long long)nseq * s.n_hb;   // unsegmented work items
     long long seg;
     if (p.num_seqs > 0) {
-        // packed: bound the longest item so no sequence dominates the makespan
-        seg = (tokens * s.n_hb + target - 1) / target;
-        seg = seg < 1024 ? 1024 : seg;
-    } else {
-        // equal-length sequences: pick the segment count with the smallest modelled
-        // makespan, in 128-token block steps of one SM.  Pass 2 runs
-        // ceil(pairs * n / SMs) rounds of items of ceil(blocks / n) blocks; pass 1
-        // (state only, about 0.65 of a pass-2 block) the same over n - 1 segments;
-        // each round costs about 1.5 blocks of fill and drain, the segment scan 2.
-        const long long pairs = (long long)p.batch * s.n_hb;
-        const long long nblk = (p.seqlen + kQ - 1) / kQ;
-        const long long sms = kPlanSMs;
-        long long best_n = 1;
-        double best = 1e300;
-        for (long long n = 1; n <= 64 && n <= nblk; ++n) {
-            const long long bps = (nblk + n - 1) / n;
-            const long long r2 = (pairs * n + sms - 1) / sms;
-            const long long r1 = n > 1 ? (pairs * (n - 1) + sms - 1) / sms : 0;
-            const double cost = (double)bps * ((double)r2 + 0.65 * (double)r1) + 1.5 * (double)(r1 + r2) +
-                                (n > 1 ? 2.0 : 0.0);
-            if (cost < best - 1e-9) {
-                best = cost;
-                best_n = n;
-            }
+        // packed: the lengths live on the device, so the model runs on rows of the
+        // average length; when it asks for cuts, segments are bounded so that no
+        // sequence dominates the makespan (about two items per SM, >= 1024 tokens)
+        const long long avg_blk = (tokens / nseq + kQ - 1) / kQ;
+        if (avg_blk < 1 || best_segment_count(items, avg_blk) == 1) {
+            seg = tokens > 0 ? tokens : kQ;
+        } else {
+            const int target = 2 * kPlanSMs;
+            seg = (tokens * s.n_hb + target - 1) / target;
+            seg = seg < 1024 ? 1024 : seg;
         }
-        seg = (nblk + best_n - 1) / best_n * kQ;
+    } else {
+        const long long nblk = (p.seqlen + kQ - 1) / kQ;
+        const long long n = best_segment_count(items, nblk > 0 ? nblk : 1);
+        seg = (nblk + n - 1) / n * kQ;
     }
     seg = (seg + kQ - 1) / kQ * kQ;
     if (seg < kQ) seg = kQ;
@@ -1109,7 +1123,7 @@ TcPlanShape plan_shape(const ssd_fwd_params &p)
     else
         s.max_segments = p.batch * (int)((p.seqlen + seg - 1) / seg);
     s.max_items = s.max_segments * s.n_hb;
-    s.segmented = p.num_seqs > 0 ? (s.seg_len < p.seqlen) : (s.seg_len < p.seqlen);
+    s.segmented = s.seg_len < p.seqlen;
     return s;
 }
 

@@ -140,8 +140,10 @@ def test_tensor_path_work_split(lib):
     assert ssd.launch_count(_tc_params(1, 128, 2, 64)) == 1
     # a 16K-token row with 32 heads: cut into segments (planner, state pass, scan, walk)
     assert ssd.launch_count(_tc_params(1, 16384, 32, 256, ngroups=8)) == 4
-    # packed variable-length batch: planner + walk, or + state pass + scan when segmented
-    assert ssd.launch_count(_tc_params(1, 32768, 48, 128, num_seqs=16)) == 4
+    # packed variable-length batch: planner + walk when there are enough items for
+    # the SMs (16 x 24 here), + state pass + scan when it must be cut (one sequence)
+    assert ssd.launch_count(_tc_params(1, 32768, 48, 128, num_seqs=16)) == 2
+    assert ssd.launch_count(_tc_params(1, 32768, 48, 128, num_seqs=1)) == 4
     assert ssd.launch_count(_tc_params(1, 512, 48, 128, num_seqs=4)) == 2
     for p in (_tc_params(8, 2048, 80, 128), _tc_params(1, 16384, 32, 256, ngroups=8),
               _tc_params(1, 32768, 48, 128, num_seqs=16)):
