@@ -65,7 +65,7 @@ extern "C" {
 typedef enum ssd_status {
     SSD_OK = 0,
     SSD_ERR_INVALID_ARG = -1,   /* null/misaligned pointer, bad dimension, workspace too small */
-    SSD_ERR_UNSUPPORTED = -2,   /* valid shape this build does not implement (see limits) */
+    SSD_ERR_UNSUPPORTED = -2,   /* valid shape the library does not implement (see limits) */
     SSD_ERR_CUDA = -3,          /* a CUDA runtime call or launch failed */
     SSD_ERR_TIMEOUT = -4,       /* device-side bounded wait gave up (status word) */
     SSD_ERR_BAD_SEQLENS = -5    /* cu_seqlens not 0 = c0 <= c1 <= ... = seqlen (status word) */
