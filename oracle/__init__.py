@@ -19,6 +19,10 @@ Structured State Space Duality":
 Readings where the pages are silent (listed in the design doc): the input is
 discretised as delta * x; A = -exp(A_log); D multiplies raw x; the initial
 state is decayed by the first token's a; packed sequences exchange no state.
+Every function here is pinned by tests/test_oracle.py (brute force, closed
+forms, invariants, hand-worked values), except for the input discretisation
+itself: the pages omit it, so that one choice (delta * x) is parity unpinned,
+a recorded reading that both formulations above share.
 """
 from __future__ import annotations
 

@@ -22,8 +22,8 @@
  *    acts as the input gate),
  *  - A = -exp(A_log) per head,
  *  - D multiplies the raw x,
- *  - the initial state is decayed by the first token's a (the listing's
- *    inclusive cumulative decay, Sec. 6 / Listing 1 step 4),
+ *  - the initial state is decayed by the first token's a (the algorithm's
+ *    state-to-output term uses an inclusive cumulative decay, Sec. 6),
  *  - packed variable-length sequences exchange no state (Sec. 8.3).
  *
  * Inputs are float32 arrays (holding the exact io-dtype values); all
