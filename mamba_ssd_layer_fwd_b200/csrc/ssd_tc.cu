@@ -123,6 +123,7 @@ struct __align__(1024) TcSmem {
     float ldec[kCsd];                  // cs_last (natural log of the block decay)
     uint64_t bc_full[2], bc_empty[2], x_full[2], x_empty[2], cs_full[kCsd], cs_empty[kCsd];
     uint64_t cb_full, cb_empty, pm_full[2], pm_empty[2], hb_full, hb_empty, xw_full[2], xw_empty[2], xw_free[2];
+    uint64_t yo_full;
     uint64_t h_ready[2], hs_full[2], y_full, yo_empty, yd_empty, drain_o, drain_s;
     uint32_t tmem_base;
     int abort;
@@ -199,6 +200,9 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
     // warp: coalesced full-line writes instead of 16-byte pieces of 32 rows.  Needs
     // two w o X slots, so the next unit's w o X pass runs meanwhile.
     constexpr bool kTmaY = !STATE_ONLY && kXwD >= 2;
+    // dstate 256 (one head per item): C bf16(H)^T is issued by the state issuer, so it
+    // never queues behind the mask-bound Pm X (+3 % there; slower with two heads)
+    constexpr bool kYoOnState = !STATE_ONLY && NST >= 256;
     constexpr int kMT = NST >= 256 ? 2 : 1;        // 128-row state tiles per head (H^T rows = n)
 
     if (tid == 0) {
@@ -224,6 +228,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
         mbar_init(&S.hb_full, 4);
         mbar_init(&S.hb_empty, 1);
         mbar_init(&S.y_full, 1);
+        mbar_init(&S.yo_full, 1);
         mbar_init(&S.yo_empty, 4);
         mbar_init(&S.yd_empty, 4);
         mbar_init(&S.drain_o, 1);
@@ -323,6 +328,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             // the whole warp runs the loop; one elected lane issues
             const bool leader = elect_one();
             const uint32_t id_h = idesc_bf16_f32(128, kP, true, true);
+            const uint32_t id_y = idesc_bf16_f32(128, kP, false, true);
             const uint32_t lbo_m = NST >= 128 ? 16384u : 0u;   // N = 64: rows 64..127 repeat rows 0..63
             bool ok = true;
             for (int c = 0; c < nblk && ok; ++c) {
@@ -349,6 +355,22 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                     if (leader) umma_commit(kTmaY ? &S.xw_free[wi] : &S.xw_empty[wi]);
                     if (leader) umma_commit(&S.h_ready[j]);
                     SSD_TRACE_EV(4, u);
+                    if (kYoOnState) {
+                        ok = mbar_wait<kInlW>(&S.hb_full, u & 1, abort) &&
+                             (u == 0 || mbar_wait<kInlW>(&S.yo_empty, (u - 1) & 1, abort));
+                        if (!ok) break;
+                        tc_fence_after();
+                        const uint64_t c0 = sdesc_sw128(smem_u32(S.bc[bs][0][0]), 16, 1024);
+                        const uint64_t h0 = sdesc_sw128(smem_u32(S.hbf), 16384, 1024);
+#pragma unroll
+                        for (int kk = 0; kk < NST / 16; ++kk) {
+                            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                            if (leader)
+                                umma_ss(tb + kColYo, desc_adv(c0, off), desc_adv(h0, kk * 2048), id_y, kk > 0);
+                        }
+                        if (leader) umma_commit(&S.hb_empty);
+                        if (leader) umma_commit(&S.yo_full);
+                    }
                 }
                 if (leader) umma_commit(&S.bc_empty[bs]);
             }
@@ -445,21 +467,23 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                 }
                 for (int j = 0; j < KH && ok; ++j) {
                     const int u = c * KH + j, xs = u & 1, pi = u & 1;
-                    // Yo = C Hbf^T
-                    ok = mbar_wait<kInlW>(&S.hb_full, u & 1, abort);
-                    SSD_TRACE_EV(14, u);
-                    ok = ok && (u == 0 || mbar_wait<kInlW>(&S.yo_empty, (u - 1) & 1, abort));
-                    SSD_TRACE_EV(17, u);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint64_t a0 = sdesc_sw128(sC, 16, 1024), b0 = sdesc_sw128(smem_u32(S.hbf), 16384, 1024);
+                    // Yo = C Hbf^T (issued by the state issuer when kYoOnState)
+                    if (!kYoOnState) {
+                        ok = mbar_wait<kInlW>(&S.hb_full, u & 1, abort);
+                        SSD_TRACE_EV(14, u);
+                        ok = ok && (u == 0 || mbar_wait<kInlW>(&S.yo_empty, (u - 1) & 1, abort));
+                        SSD_TRACE_EV(17, u);
+                        if (!ok) break;
+                        tc_fence_after();
+                        const uint64_t a0 = sdesc_sw128(sC, 16, 1024), b0 = sdesc_sw128(smem_u32(S.hbf), 16384, 1024);
 #pragma unroll
-                    for (int kk = 0; kk < NST / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                        if (leader) umma_ss(tb + kColYo, desc_adv(a0, off), desc_adv(b0, kk * 2048), id_y, kk > 0);
+                        for (int kk = 0; kk < NST / 16; ++kk) {
+                            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                            if (leader) umma_ss(tb + kColYo, desc_adv(a0, off), desc_adv(b0, kk * 2048), id_y, kk > 0);
+                        }
+                        if (leader) umma_commit(&S.hb_empty);
+                        SSD_TRACE_EV(3, u);
                     }
-                    if (leader) umma_commit(&S.hb_empty);
-                    SSD_TRACE_EV(3, u);
                     // the next block's CB runs while the mask warps finish this block's last head
                     if (kSt > 1 && j == KH - 1 && c + 1 < nblk) {
                         ok = issue_cb(c + 1);
@@ -708,6 +732,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
         auto epilogue = [&](int v) -> bool {
             const int c = v / KH, j = v % KH, slot = v % kCsd;
             if (!mbar_wait<kInlW>(&S.y_full, v & 1, abort)) return false;
+            if (kYoOnState && !mbar_wait<kInlW>(&S.yo_full, v & 1, abort)) return false;
             tc_fence_after();
             if (warp == 12 && lane == 0) SSD_TRACE_EV(12, v);
             const int valid = min(kQ, it.len - c * kQ);
