@@ -16,6 +16,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import re
 import os
 import signal
 import statistics
@@ -67,12 +68,23 @@ def algorithmic_flops(inp: dict) -> int:
     return int(tokens * (H * (4 * P * N + Q * P) + G * Q * N))
 
 
+def _code_only(text: str) -> str:
+    """CUDA/C++ source without comments and with whitespace collapsed, so that
+    editing a comment does not change the hash (the sources contain no comment
+    markers inside string literals)."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_hash() -> str:
+    """Hash of the library's CUDA sources (code only): the committed ncu
+    traffic figures apply while it matches."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mamba_ssd_layer_fwd_b200", "csrc")
     for fn in sorted(os.listdir(csrc)):
         if fn.endswith((".cu", ".cuh")):
-            h.update(open(os.path.join(csrc, fn), "rb").read())
+            h.update(fn.encode() + b"\0" + _code_only(open(os.path.join(csrc, fn)).read()).encode() + b"\0")
     return h.hexdigest()[:16]
 
 

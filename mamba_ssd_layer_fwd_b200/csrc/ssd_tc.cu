@@ -25,17 +25,20 @@
 //
 // Warp roles (16 warps; warp w runs on SM sub-partition w % 4 and may only
 // touch TMEM lanes 32*(w%4) .. +31): 0 cumsum, 1 UMMA issuer for the state
-// path (H += B^T (w o X)), 2 TMA producer, 3 UMMA issuer for the output
-// path (CB, C Hbf^T, Pm X) + TMEM owner, 4-7 and 10-11 mask (the causal
-// work of rows 96-127 is four times that of rows 0-31, so sub-partitions
-// 0-1 also get the w o X pass, warps 8-9), 12-15 state rescale + output
-// epilogue.  Two issuers keep the state and output paths from waiting on
+// path (H += B^T (w o X); also C Hbf^T when dstate is 256), 2 TMA producer,
+// 3 UMMA issuer for the output path (CB, C Hbf^T, Pm X) + TMEM owner, 4-7
+// and 10-11 mask (the causal work of rows 96-127 is four times that of rows
+// 0-31, so sub-partitions 0-1 also get the w o X pass, warps 8-9), 12-15
+// state rescale + output epilogue.  Two issuers keep the state and output paths from waiting on
 // each other.  Every mbarrier wait is bounded (2 s); on a timeout the CTA
 // records SSD_ERR_TIMEOUT in the status word, drains, frees TMEM and exits.
 //
-// When there are too few (sequence, head block) pairs to fill the GPU, each
-// sequence is cut into segments.  A first launch of the same kernel in
-// state-only mode computes every non-final segment's end state from zero;
+// Equal-length rows that need no cuts take their work item from the block
+// index (no planner kernel); two-head items left over after whole waves of
+// the SMs run as one-head items in a second launch.  When there are too few
+// (sequence, head block) pairs to fill the GPU, each sequence is cut into
+// segments.  A first launch of the same kernel in state-only mode computes
+// every non-final segment's end state from zero;
 // a scan kernel turns those into each segment's entering state; the full
 // walk then starts every segment from its true state (Sec. 8.2: state
 // passing between pieces of a sequence).
