@@ -23,3 +23,17 @@ def test_reference_arm_prints_one_contract_line():
     assert d["config"]["workload"] == "small_bf16"
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+
+
+def test_traffic_figures_follow_code_not_comments():
+    """The committed ncu traffic applies while the CUDA code (not its comments)
+    is unchanged."""
+    sys.path.insert(0, ROOT)
+    import bench
+    a = "int f() { return 1; } // one\n/* block\ncomment */ int g;"
+    b = "int f() {  return 1; }   // another comment\nint g;"
+    c = "int f() { return 2; } // one\nint g;"
+    assert bench._code_only(a) == bench._code_only(b)
+    assert bench._code_only(a) != bench._code_only(c)
+    h = bench.kernel_source_hash()
+    assert len(h) == 16 and h == bench.kernel_source_hash()
