@@ -16,7 +16,7 @@ Structured State Space Duality":
   (lower triangle) explicitly and multiply. numpy, tiny sizes only. It pins the
   recurrence.
 
-Readings where the pages are silent (listed in the design doc): the input is
+Readings where the pages are silent (the CUDA path makes the same ones): the input is
 discretised as delta * x; A = -exp(A_log); D multiplies raw x; the initial
 state is decayed by the first token's a; packed sequences exchange no state.
 Every function here is pinned by tests/test_oracle.py (brute force, closed

@@ -17,7 +17,7 @@
  *       y[t, h, :] = state @ C[t, g, :] + D[h] * x[t, h, :]
  *     final_states[s, h] = state
  *
- * Readings of points the pages leave open (each is recorded in the design doc):
+ * Readings of points the pages leave open (the same in the CUDA path):
  *  - the input is discretised as delta * x (Sec. 2.1 omits the rule; delta
  *    acts as the input gate),
  *  - A = -exp(A_log) per head,

@@ -49,14 +49,18 @@ def rel_err(a, b):
 
 # ---------------------------------------------------------------- golden values
 
+_EXPR = {"log(ln(2)/2)": math.log(math.log(2) / 2), "0": 0.0, "30": 30.0,
+         "log(ln(2))": math.log(math.log(2)), "ln(3)": math.log(3.0), "-ln(3)": -math.log(3.0)}
+
+
 def _golden_inp(case):
-    T = len(case["dt"])
+    dt = [_EXPR[e] for e in case["dt_expr"]] if "dt_expr" in case else case["dt"]
+    T = len(dt)
     P, N = case["P"], case["N"]
-    A_log = {"log(ln(2)/2)": math.log(math.log(2) / 2), "0": 0.0,
-             "log(ln(2))": math.log(math.log(2))}[case["A_log_expr"]]
+    A_log = _EXPR[case["A_log_expr"]]
     inp = {
         "x": np.array(case["x"], dtype=np.float32).reshape(1, T, 1, P),
-        "dt": np.array(case["dt"], dtype=np.float32).reshape(1, T, 1),
+        "dt": np.array(dt, dtype=np.float32).reshape(1, T, 1),
         "A_log": np.array([A_log], dtype=np.float32),
         "B": np.array(case["B"], dtype=np.float32).reshape(1, T, 1, N),
         "C": np.array(case["C"], dtype=np.float32).reshape(1, T, 1, N),
@@ -68,22 +72,41 @@ def _golden_inp(case):
     return inp
 
 
-@pytest.mark.parametrize("idx", [0, 1, 2])
+@pytest.mark.parametrize("idx", [0, 1, 2, 3, 4])
 def test_golden_hand_worked(idx):
-    """Hand-worked values of the recurrence (tests/golden/scalar_recurrence.json)."""
+    """Hand-worked values of the recurrence (tests/golden/scalar_recurrence.json).
+    Cases 3 and 4 pin the discretisation delta = softplus(dt) = log(1 + e^dt)
+    away from dt = 0 (both signs, and |dt| up to 1000 where the naive form
+    overflows): a sign flip or a dropped max(dt, 0) term fails them."""
     case = json.load(open(os.path.join(GOLDEN, "scalar_recurrence.json")))["cases"][idx]
     inp = _golden_inp(case)
     y, fin = oracle.recurrence(inp)
-    ln2 = math.log(2.0)
+    ln2, ln3 = math.log(2.0), math.log(3.0)
     if "y_ln2" in case:
         want_y = np.array([c0 + c1 * ln2 for c0, c1 in case["y_ln2"]])
         want_f = case["final_ln2"][0] + case["final_ln2"][1] * ln2
+    elif "y_ln23" in case:
+        want_y = np.array([c0 + c1 * ln2 + c2 * ln3 for c0, c1, c2 in case["y_ln23"]])
+        want_f = case["final_ln23"][0] + case["final_ln23"][1] * ln2 + case["final_ln23"][2] * ln3
     else:
         want_y = np.array(case["y"], dtype=np.float64)
         want_f = np.array(case["final"], dtype=np.float64)
-    # A_log is stored in float32, so a = 1/2 holds to ~1e-7 relative
-    np.testing.assert_allclose(y.reshape(want_y.shape), want_y, rtol=2e-6, atol=1e-6)
-    np.testing.assert_allclose(fin.reshape(np.shape(want_f)), want_f, rtol=2e-6, atol=1e-6)
+    # A_log and dt are stored in float32, so a = 1/2 (or ln 3) holds to ~1e-7 relative
+    rtol = case.get("rtol", 2e-6)
+    np.testing.assert_allclose(y.reshape(want_y.shape), want_y, rtol=rtol, atol=1e-6)
+    np.testing.assert_allclose(fin.reshape(np.shape(want_f)), want_f, rtol=rtol, atol=1e-6)
+
+
+def test_discretize_softplus_matches_logaddexp():
+    """delta = softplus(r) = log(e^0 + e^r): numpy's logaddexp is an independent
+    evaluation of the same definition (Sec. 2.1 discretisation step size)."""
+    r = np.array([-1000.0, -30.0, -5.0, -math.log(3.0), -1e-3, 0.0, 1e-3, math.log(3.0), 2.0, 30.0, 1000.0])
+    inp = {"x": np.zeros((1, r.size, 1, 1)), "dt": r.reshape(1, -1, 1), "A_log": np.array([0.0]),
+           "dt_softplus": True}
+    delta, a = oracle.discretize(inp)
+    want = np.logaddexp(0.0, r)
+    np.testing.assert_allclose(delta[:, 0], want, rtol=1e-15, atol=0.0)
+    np.testing.assert_allclose(a[:, 0], np.exp(-want), rtol=1e-15, atol=0.0)
 
 
 # ---------------------------------------------------- brute-force quadratic form
