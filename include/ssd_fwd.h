@@ -54,7 +54,7 @@
 extern "C" {
 #endif
 
-#define SSD_ABI_VERSION 1
+#define SSD_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define SSD_API __attribute__((visibility("default")))
@@ -102,11 +102,6 @@ typedef struct ssd_fwd_params {
     ssd_dtype io_dtype;
     int dt_softplus;            /* 1: delta = softplus(dt); 0: delta = dt (must be >= 0) */
     ssd_path path;
-    void *prof_begin;           /* optional cudaEvent_t recorded on `stream` right before the main kernel */
-    void *prof_end;             /* optional cudaEvent_t recorded right after it */
-    int debug_withhold_load;    /* testing only, 0 normally: nonzero makes the tensor-core path withhold
-                                   the first x tile of work item 0, so that item's bounded waits run out
-                                   and the call reports SSD_ERR_TIMEOUT through ssd_get_status */
 } ssd_fwd_params;
 
 /* Bytes of device workspace ssd_fwd needs for these parameters (0 on invalid
@@ -125,6 +120,28 @@ SSD_API ssd_status ssd_fwd(const ssd_fwd_params *p,
                    void *y, float *final_states,
                    void *workspace, size_t workspace_bytes, void *stream);
 
+/* Measurement and failure-injection hooks for ssd_fwd_instrumented (profiling
+ * tools and the library's own tests; ordinary callers use ssd_fwd). */
+typedef struct ssd_fwd_instrumentation {
+    void *ev_begin;             /* cudaEvent_t or NULL: recorded on `stream` before the first compute
+                                   kernel (after the work planner / status reset) */
+    void *ev_main;              /* cudaEvent_t or NULL: recorded before the kernel that writes y (equals
+                                   ev_begin unless a state-only pass and segment scan run first) */
+    void *ev_end;               /* cudaEvent_t or NULL: recorded after the last kernel */
+    int withhold_first_tile;    /* 0 normally; nonzero makes the tensor-core path withhold the first x tile
+                                   of work item 0, so that item's bounded waits run out and the call reports
+                                   SSD_ERR_TIMEOUT through ssd_get_status (no fault, the context survives) */
+} ssd_fwd_instrumentation;
+
+/* ssd_fwd with instrumentation; `ins` may be NULL (then identical to ssd_fwd). */
+SSD_API ssd_status ssd_fwd_instrumented(const ssd_fwd_params *p,
+                   const void *x, const void *dt, const float *A_log,
+                   const void *B, const void *C, const float *D,
+                   const float *initial_states, const int32_t *cu_seqlens,
+                   void *y, float *final_states,
+                   void *workspace, size_t workspace_bytes, void *stream,
+                   const ssd_fwd_instrumentation *ins);
+
 /* Size of the fixed scratch array behind ssd_fwd_noalloc: 16 MiB of device
  * memory on every GPU that loads this library, held until the process exits. */
 #define SSD_NOALLOC_SCRATCH_BYTES (16u << 20)
@@ -141,7 +158,10 @@ SSD_API ssd_status ssd_fwd(const ssd_fwd_params *p,
  *     more workspace than SSD_NOALLOC_SCRATCH_BYTES (ssd_fwd_workspace_size).
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
  *   - The first call on a device looks up the array's address with that
- *     device current; make it before any stream capture.
+ *     device current; make it before any stream capture.  The address is kept
+ *     for the life of the process: after cudaDeviceReset (or any other
+ *     teardown of the device's primary context) it is stale, and this entry
+ *     point must not be called again on that device.
  *   - Every call shares the array.  The kernels clear what must start at zero
  *     and overwrite the rest before reading it, but calls that overlap on the
  *     GPU (other streams, other threads on the same device) race on it.

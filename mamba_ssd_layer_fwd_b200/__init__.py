@@ -22,8 +22,8 @@ import threading
 from typing import Optional
 
 __all__ = [
-    "ssd_fwd", "ssd_decode_step", "SsdParams", "SsdStepParams", "workspace_size", "launch_count", "resolved_path", "library",
-    "library_path", "STATUS", "PATHS", "SsdError",
+    "ssd_fwd", "ssd_decode_step", "SsdParams", "SsdStepParams", "SsdInstrumentation", "make_instrumentation", "workspace_size",
+    "launch_count", "resolved_path", "library", "library_path", "STATUS", "PATHS", "SsdError",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -36,7 +36,7 @@ STATUS = {0: "SSD_OK", -1: "SSD_ERR_INVALID_ARG", -2: "SSD_ERR_UNSUPPORTED", -3:
 PATHS = {"auto": 0, "simt": 1, "tensor": 2}
 DTYPES = {"f32": 0, "bf16": 1}
 
-EXPORTED = ("ssd_fwd", "ssd_decode_step", "ssd_fwd_workspace_size", "ssd_get_status", "ssd_fwd_launch_count",
+EXPORTED = ("ssd_fwd", "ssd_fwd_instrumented", "ssd_decode_step", "ssd_fwd_workspace_size", "ssd_get_status", "ssd_fwd_launch_count",
             "ssd_fwd_resolved_path", "ssd_status_string", "ssd_abi_version")
 
 
@@ -52,8 +52,15 @@ class SsdParams(ctypes.Structure):
         ("headdim", ctypes.c_int), ("dstate", ctypes.c_int), ("ngroups", ctypes.c_int),
         ("chunk_len", ctypes.c_int), ("num_seqs", ctypes.c_int), ("io_dtype", ctypes.c_int),
         ("dt_softplus", ctypes.c_int), ("path", ctypes.c_int),
-        ("prof_begin", ctypes.c_void_p), ("prof_end", ctypes.c_void_p),
-        ("debug_withhold_load", ctypes.c_int),
+    ]
+
+
+class SsdInstrumentation(ctypes.Structure):
+    """ssd_fwd_instrumentation: CUDA events recorded around the compute
+    kernels, and the failure-injection switch used by the timeout test."""
+    _fields_ = [
+        ("ev_begin", ctypes.c_void_p), ("ev_main", ctypes.c_void_p), ("ev_end", ctypes.c_void_p),
+        ("withhold_first_tile", ctypes.c_int),
     ]
 
 
@@ -81,6 +88,9 @@ def library():
             vp, sz, i32, pp = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.POINTER(SsdParams)
             lib.ssd_fwd.restype = i32
             lib.ssd_fwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+            lib.ssd_fwd_instrumented.restype = i32
+            lib.ssd_fwd_instrumented.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
+                                                 ctypes.POINTER(SsdInstrumentation)]
             lib.ssd_decode_step.restype = i32
             lib.ssd_decode_step.argtypes = [ctypes.POINTER(SsdStepParams), vp, vp, vp, vp, vp, vp, vp, vp, vp]
             lib.ssd_fwd_workspace_size.restype = sz
@@ -107,11 +117,16 @@ def _status_string(code: int) -> str:
 
 
 def make_params(*, batch, seqlen, nheads, headdim, dstate, ngroups, chunk_len, num_seqs=0,
-                io_dtype="bf16", dt_softplus=True, path="auto", prof_begin=None,
-                prof_end=None) -> SsdParams:
+                io_dtype="bf16", dt_softplus=True, path="auto") -> SsdParams:
     return SsdParams(int(batch), int(seqlen), int(nheads), int(headdim), int(dstate), int(ngroups),
                      int(chunk_len), int(num_seqs), DTYPES[io_dtype], int(bool(dt_softplus)),
-                     PATHS[path], prof_begin, prof_end, 0)
+                     PATHS[path])
+
+
+def make_instrumentation(events=None, withhold_first_tile=False) -> SsdInstrumentation:
+    """events = (begin, main, end) torch.cuda.Event objects (or None each)."""
+    ev = [None, None, None] if events is None else [None if e is None else int(e.cuda_event) for e in events]
+    return SsdInstrumentation(ev[0], ev[1], ev[2], int(bool(withhold_first_tile)))
 
 
 def workspace_size(params: SsdParams) -> int:
@@ -138,8 +153,7 @@ def _stream_handle(stream) -> Optional[int]:
     return int(stream.cuda_stream) or None
 
 
-def params_for(x, B, chunk_len: int, cu_seqlens=None, dt_softplus=True, path="auto",
-               prof_events=None) -> SsdParams:
+def params_for(x, B, chunk_len: int, cu_seqlens=None, dt_softplus=True, path="auto") -> SsdParams:
     import torch
     if x.dtype == torch.bfloat16:
         io = "bf16"
@@ -150,25 +164,22 @@ def params_for(x, B, chunk_len: int, cu_seqlens=None, dt_softplus=True, path="au
     b, T, H, P = x.shape
     G, N = B.shape[2], B.shape[3]
     nseq = 0 if cu_seqlens is None else int(cu_seqlens.numel()) - 1
-    pb = pe = None
-    if prof_events is not None:
-        pb, pe = (int(e.cuda_event) for e in prof_events)
     return make_params(batch=b, seqlen=T, nheads=H, headdim=P, dstate=N, ngroups=G,
                        chunk_len=chunk_len, num_seqs=nseq, io_dtype=io, dt_softplus=dt_softplus,
-                       path=path, prof_begin=pb, prof_end=pe)
+                       path=path)
 
 
 def ssd_fwd(x, dt, A_log, B, C, D=None, chunk_len: int = 256, initial_states=None,
             cu_seqlens=None, dt_softplus: bool = True, return_final_states: bool = False,
             y=None, final_states=None, workspace=None, stream=None, path: str = "auto",
-            prof_events=None, check_status: bool = False):
+            instrumentation: Optional[SsdInstrumentation] = None, check_status: bool = False):
     """SSD forward on the GPU through the C ABI. Returns y, or (y, final_states)
     when `return_final_states` is true (or `final_states` is given).
 
     x, dt, B, C share the io dtype (bfloat16 or float32); A_log, D,
     initial_states are float32; cu_seqlens is int32. Outputs and the workspace
-    are allocated with torch on x's device unless passed in. `prof_events` =
-    (begin, end) torch.cuda.Event pair recorded around the main kernel.
+    are allocated with torch on x's device unless passed in. `instrumentation`
+    (make_instrumentation) routes the call through ssd_fwd_instrumented.
     """
     import torch
     lib = library()
@@ -185,7 +196,7 @@ def ssd_fwd(x, dt, A_log, B, C, D=None, chunk_len: int = 256, initial_states=Non
         raise ValueError("cu_seqlens must be a contiguous int32 tensor")
     if x.dim() != 4 or dt.shape != x.shape[:3] or B.shape != C.shape or B.shape[:2] != x.shape[:2]:
         raise ValueError("shape mismatch between x, dt, B, C")
-    p = params_for(x, B, chunk_len, cu_seqlens, dt_softplus, path, prof_events)
+    p = params_for(x, B, chunk_len, cu_seqlens, dt_softplus, path)
     b, T, H, P = x.shape
     N = B.shape[3]
     nseq = p.num_seqs if p.num_seqs > 0 else b
@@ -204,9 +215,13 @@ def ssd_fwd(x, dt, A_log, B, C, D=None, chunk_len: int = 256, initial_states=Non
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     st = _stream_handle(stream)
-    rc = lib.ssd_fwd(ctypes.byref(p), _ptr(x), _ptr(dt), _ptr(A_log), _ptr(B), _ptr(C), _ptr(D),
-                     _ptr(initial_states), _ptr(cu_seqlens), _ptr(y), _ptr(final_states),
-                     _ptr(workspace), workspace.numel() * workspace.element_size(), st)
+    args = (ctypes.byref(p), _ptr(x), _ptr(dt), _ptr(A_log), _ptr(B), _ptr(C), _ptr(D),
+            _ptr(initial_states), _ptr(cu_seqlens), _ptr(y), _ptr(final_states),
+            _ptr(workspace), workspace.numel() * workspace.element_size(), st)
+    if instrumentation is None:
+        rc = lib.ssd_fwd(*args)
+    else:
+        rc = lib.ssd_fwd_instrumented(*args, ctypes.byref(instrumentation))
     if rc != 0:
         raise SsdError(rc, "ssd_fwd")
     if check_status:

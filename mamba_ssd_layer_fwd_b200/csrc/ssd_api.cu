@@ -139,6 +139,15 @@ ssd_status ssd_fwd(const ssd_fwd_params *p, const void *x, const void *dt, const
                    const int32_t *cu_seqlens, void *y, float *final_states, void *workspace,
                    size_t workspace_bytes, void *stream)
 {
+    return ssd_fwd_instrumented(p, x, dt, A_log, B, C, D, initial_states, cu_seqlens, y, final_states, workspace,
+                                workspace_bytes, stream, nullptr);
+}
+
+ssd_status ssd_fwd_instrumented(const ssd_fwd_params *p, const void *x, const void *dt, const float *A_log,
+                                const void *B, const void *C, const float *D, const float *initial_states,
+                                const int32_t *cu_seqlens, void *y, float *final_states, void *workspace,
+                                size_t workspace_bytes, void *stream, const ssd_fwd_instrumentation *instr)
+{
     try {
         const ssd_status v = validate(p);
         if (v != SSD_OK) return v;
@@ -175,8 +184,13 @@ ssd_status ssd_fwd(const ssd_fwd_params *p, const void *x, const void *dt, const
         d.tokens = p->batch * p->seqlen;
         d.dt_softplus = p->dt_softplus;
 
-        cudaEvent_t pb = static_cast<cudaEvent_t>(p->prof_begin);
-        cudaEvent_t pe = static_cast<cudaEvent_t>(p->prof_end);
+        Instr ins;
+        if (instr) {
+            ins.begin = static_cast<cudaEvent_t>(instr->ev_begin);
+            ins.main = static_cast<cudaEvent_t>(instr->ev_main);
+            ins.end = static_cast<cudaEvent_t>(instr->ev_end);
+            ins.withhold_first_tile = instr->withhold_first_tile;
+        }
         cudaError_t e;
         if (path == SSD_PATH_SIMT) {
             // the chunk table kernel also clears the status word
@@ -190,7 +204,7 @@ ssd_status ssd_fwd(const ssd_fwd_params *p, const void *x, const void *dt, const
             a.dv = reinterpret_cast<float *>(ws + L.dv);
             a.states = reinterpret_cast<float *>(ws + L.states);
             a.bf16 = p->io_dtype == SSD_DTYPE_BF16;
-            e = launch_simt(plan, d, a, st, pb, pe);
+            e = launch_simt(plan, d, a, st, ins);
         } else {
             TcArgs a;
             a.x = x; a.dt = dt; a.B = B; a.C = C;
@@ -199,7 +213,7 @@ ssd_status ssd_fwd(const ssd_fwd_params *p, const void *x, const void *dt, const
             a.y = y; a.final_states = final_states;
             a.scratch = ws + L.tc;
             a.scratch_bytes = L.total - L.tc;
-            e = launch_tc(*p, plan, d, a, st, pb, pe);
+            e = launch_tc(*p, plan, d, a, st, ins);
         }
         return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
     } catch (const std::bad_alloc &) {

@@ -77,6 +77,13 @@ __device__ __forceinline__ float softplus_f32(float r)
     return fmaxf(r, 0.0f) + log1pf(__expf(-fabsf(r)));
 }
 
+// Events and the failure-injection switch of ssd_fwd_instrumented (all null /
+// zero for plain ssd_fwd).
+struct Instr {
+    cudaEvent_t begin = nullptr, main = nullptr, end = nullptr;
+    int withhold_first_tile = 0;
+};
+
 // Host-side launchers (one per translation unit).
 cudaError_t launch_build_plan(const Plan &plan, const int32_t *cu_seqlens, int batch, int seqlen,
                               int chunk_len, cudaStream_t stream);
@@ -90,6 +97,6 @@ struct SimtArgs {
     int bf16;
 };
 cudaError_t launch_simt(const Plan &plan, const Dims &d, const SimtArgs &a, cudaStream_t stream,
-                        cudaEvent_t prof_begin, cudaEvent_t prof_end);
+                        const Instr &ins);
 
 }  // namespace ssd

@@ -281,8 +281,7 @@ size_t scan_smem(const Dims &d)
 }
 
 template <typename T>
-cudaError_t launch_typed(const Plan &plan, const Dims &d, const SimtArgs &a, cudaStream_t st,
-                         cudaEvent_t pb, cudaEvent_t pe)
+cudaError_t launch_typed(const Plan &plan, const Dims &d, const SimtArgs &a, cudaStream_t st, const Instr &ins)
 {
     const T *x = static_cast<const T *>(a.x);
     const T *dt = static_cast<const T *>(a.dt);
@@ -290,6 +289,7 @@ cudaError_t launch_typed(const Plan &plan, const Dims &d, const SimtArgs &a, cud
     const T *Cm = static_cast<const T *>(a.C);
     T *y = static_cast<T *>(a.y);
     const dim3 gc(plan.max_chunks, d.H);
+    if (ins.begin) cudaEventRecord(ins.begin, st);
     chunk_cumsum_kernel<T><<<gc, d.Q, 0, st>>>(plan, d, dt, a.A_log, a.cs, a.dv);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -308,16 +308,16 @@ cudaError_t launch_typed(const Plan &plan, const Dims &d, const SimtArgs &a, cud
     e = cudaFuncSetAttribute(chunk_scan_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sc);
     if (e != cudaSuccess) return e;
     const dim3 gs(plan.max_chunks, d.H, (d.Q + kTile - 1) / kTile);
-    if (pb) cudaEventRecord(pb, st);
+    if (ins.main) cudaEventRecord(ins.main, st);
     chunk_scan_kernel<T><<<gs, kThreads, sc, st>>>(plan, d, x, Bm, Cm, a.D, a.cs, a.dv, a.states, y);
-    if (pe) cudaEventRecord(pe, st);
+    if (ins.end) cudaEventRecord(ins.end, st);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_simt(const Plan &plan, const Dims &d, const SimtArgs &a, cudaStream_t stream,
-                        cudaEvent_t prof_begin, cudaEvent_t prof_end)
+                        const Instr &ins)
 {
     if (plan.max_chunks == 0) {
         // nothing to compute; final states still equal the initial states
@@ -326,8 +326,7 @@ cudaError_t launch_simt(const Plan &plan, const Dims &d, const SimtArgs &a, cuda
             state_passing_kernel<<<gp, kThreads, 0, stream>>>(plan, d, a.cs, a.states, a.init, a.final_states);
         return cudaGetLastError();
     }
-    return a.bf16 ? launch_typed<__nv_bfloat16>(plan, d, a, stream, prof_begin, prof_end)
-                  : launch_typed<float>(plan, d, a, stream, prof_begin, prof_end);
+    return a.bf16 ? launch_typed<__nv_bfloat16>(plan, d, a, stream, ins) : launch_typed<float>(plan, d, a, stream, ins);
 }
 
 }  // namespace ssd

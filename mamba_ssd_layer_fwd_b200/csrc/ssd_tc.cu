@@ -935,10 +935,14 @@ tc_plan_kernel(const int32_t *__restrict__ cu_seqlens, int nseq, int seqlen, int
     }
     __syncthreads();
     if (s_bad) {
+        // no work item and no segment chain: the later kernels of this call read
+        // nothing from a previous call's tables
         if (tid == 0) {
             set_status(status, kDevBadSeqlens);
             *count = 0;
         }
+        if (seqseg)
+            for (int i = tid; i < nseq; i += 1024) seqseg[i] = -1;
         return;
     }
     for (int base = 0; base < nseq; base += 1024) {
@@ -1019,12 +1023,15 @@ tc_plan_kernel(const int32_t *__restrict__ cu_seqlens, int nseq, int seqlen, int
 // place over the pass-1 end states.
 __global__ void __launch_bounds__(256)
 tc_seg_scan_kernel(const TcItem *__restrict__ items, const int *__restrict__ seqseg, int n_hb, float *segstate,
-                   const float *__restrict__ seglogdec, const float *__restrict__ init, int H, int PN)
+                   const float *__restrict__ seglogdec, const float *__restrict__ init, int H, int PN,
+                   const int *__restrict__ count, int max_segments)
 {
     // grid: (sequences, H, ceil(PN / 256)); only sequences cut into two or more segments work
     const int gs = seqseg[blockIdx.x];
-    if (gs < 0) return;
+    // a plan the planner rejected (malformed cu_seqlens) has no items
+    if (gs < 0 || gs >= max_segments || (long long)gs * n_hb >= *count) return;
     const TcItem it = items[(size_t)gs * n_hb];
+    if (gs + it.nseg > max_segments) return;
     const int h = blockIdx.y;
     const int e = blockIdx.z * 256 + threadIdx.x;
     if (e >= PN) return;
@@ -1240,7 +1247,7 @@ int tc_launch_count(const ssd_fwd_params &p)
 }
 
 cudaError_t launch_tc(const ssd_fwd_params &p, const Plan &plan, const Dims &d, const TcArgs &a,
-                      cudaStream_t stream, cudaEvent_t prof_begin, cudaEvent_t prof_end)
+                      cudaStream_t stream, const Instr &ins)
 {
     const TcPlanShape s = plan_shape(p);
     char *ws = static_cast<char *>(a.scratch);
@@ -1299,16 +1306,18 @@ cudaError_t launch_tc(const ssd_fwd_params &p, const Plan &plan, const Dims &d, 
     prm.N = p.dstate;
     prm.heads_per_group = d.heads_per_group;
     prm.dt_softplus = p.dt_softplus;
-    prm.withhold_x0 = p.debug_withhold_load != 0;
+    prm.withhold_x0 = ins.withhold_first_tile != 0;
 
+    if (ins.begin) cudaEventRecord(ins.begin, stream);
     if (s.segmented) {
         e = launch_walk_any<true>(p.dstate, s.KH, s.max_items, mX, mB, mC, mY, prm, stream);
         if (e != cudaSuccess) return e;
         const dim3 gs(nseq, p.nheads, (PN + 255) / 256);
-        tc_seg_scan_kernel<<<gs, 256, 0, stream>>>(items, seqseg, s.n_hb, segstate, seglogdec, a.init, p.nheads, PN);
+        tc_seg_scan_kernel<<<gs, 256, 0, stream>>>(items, seqseg, s.n_hb, segstate, seglogdec, a.init, p.nheads, PN,
+                                                   plan.count, s.max_segments);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    if (prof_begin) cudaEventRecord(prof_begin, stream);
+    if (ins.main) cudaEventRecord(ins.main, stream);
     const int split = direct_split(p, s);
     if (split < 0) {
         e = launch_walk_any<false>(p.dstate, s.KH, s.max_items, mX, mB, mC, mY, prm, stream);
@@ -1322,7 +1331,7 @@ cudaError_t launch_tc(const ssd_fwd_params &p, const Plan &plan, const Dims &d, 
             e = launch_walk_any<false>(p.dstate, 1, tail.n_items, mX, mB, mC, mY, tail, stream);
         }
     }
-    if (prof_end) cudaEventRecord(prof_end, stream);
+    if (ins.end) cudaEventRecord(ins.end, stream);
     return e;
 }
 

@@ -19,6 +19,6 @@ bool tc_supported(const ssd_fwd_params &p);
 size_t tc_workspace_bytes(const ssd_fwd_params &p);
 int tc_launch_count(const ssd_fwd_params &p);
 cudaError_t launch_tc(const ssd_fwd_params &p, const Plan &plan, const Dims &d, const TcArgs &a,
-                      cudaStream_t stream, cudaEvent_t prof_begin, cudaEvent_t prof_end);
+                      cudaStream_t stream, const Instr &ins);
 
 }  // namespace ssd

@@ -34,7 +34,7 @@ def test_exports_every_declared_symbol(lib):
     assert "ssd_fwd" in names and "ssd_fwd_workspace_size" in names
     for n in names:
         assert hasattr(lib, n), f"{n} declared in include/ but not exported"
-    assert lib.ssd_abi_version() == 1
+    assert lib.ssd_abi_version() == 2
 
 
 def test_only_abi_symbols_exported(lib):

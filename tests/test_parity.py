@@ -152,14 +152,14 @@ def test_device_wait_timeout_reported():
     inp = small_inputs(batch=1, seqlen=512, H=2, P=64, N=64, G=1, Q=256, init=False, seed=12)
     t = to_device(inp)
     p = ssd.params_for(t["x"], t["B"], 256, None, True, "tensor")
-    p.debug_withhold_load = 1
+    ins = ssd.make_instrumentation(withhold_first_tile=True)
     lib = ssd.library()
     ws = torch.empty(ssd.workspace_size(p), dtype=torch.uint8, device="cuda")
     y = torch.empty_like(t["x"])
     st = torch.cuda.current_stream().cuda_stream or None
-    rc = lib.ssd_fwd(ctypes.byref(p), t["x"].data_ptr(), t["dt"].data_ptr(), t["A_log"].data_ptr(),
-                     t["B"].data_ptr(), t["C"].data_ptr(), t["D"].data_ptr(), None, None, y.data_ptr(), None,
-                     ws.data_ptr(), ws.numel(), st)
+    rc = lib.ssd_fwd_instrumented(ctypes.byref(p), t["x"].data_ptr(), t["dt"].data_ptr(), t["A_log"].data_ptr(),
+                                  t["B"].data_ptr(), t["C"].data_ptr(), t["D"].data_ptr(), None, None, y.data_ptr(),
+                                  None, ws.data_ptr(), ws.numel(), st, ctypes.byref(ins))
     assert rc == 0
     assert lib.ssd_get_status(ws.data_ptr(), st) == -4      # SSD_ERR_TIMEOUT
     # the same context keeps working
