@@ -58,13 +58,15 @@ def algorithmic_bytes(inp: dict) -> int:
     return int(n)
 
 
-def algorithmic_flops(inp: dict) -> int:
+def algorithmic_flops(inp: dict, block_len: int) -> int:
     """Useful (causal-halved) FLOPs of the chunked algorithm per forward:
-    per token H * (4PN + Q*P) + G * Q * N."""
+    per token H * (4PN + Q*P) + G * Q * N, with Q the diagonal-block length the
+    path actually evaluates (128 on the tensor-core path, chunk_len on the
+    SIMT path)."""
     x, B = inp["x"], inp["B"]
     tokens = x.shape[0] * x.shape[1]
     H, P, G, N = x.shape[2], x.shape[3], B.shape[2], B.shape[3]
-    Q = inp["chunk_len"]
+    Q = block_len
     return int(tokens * (H * (4 * P * N + Q * P) + G * Q * N))
 
 
@@ -263,6 +265,129 @@ def run_reference(args):
     return 0
 
 
+def _device_inputs(inp, dev):
+    """Pinned host copies and device copies of a workload's inputs."""
+    import torch
+    io = torch.bfloat16 if inp["io_dtype"] == "bf16" else torch.float32
+    host = {k: torch.from_numpy(inp[k]).to(io).pin_memory() for k in ("x", "dt", "B", "C")}
+    for k in ("A_log", "D", "initial_states"):
+        host[k] = None if inp[k] is None else torch.from_numpy(inp[k]).pin_memory()
+    host["cu_seqlens"] = None if inp["cu_seqlens"] is None else torch.from_numpy(inp["cu_seqlens"]).pin_memory()
+    d = {k: (None if v is None else v.to(dev)) for k, v in host.items()}
+    return host, d
+
+
+def _stats(v):
+    return {"mean": statistics.mean(v), "median": statistics.median(v), "min": min(v)}
+
+
+class Forward:
+    """One workload resident on the device, with its outputs, workspace and a
+    step() that runs one ssd_fwd with events around the compute kernels."""
+
+    def __init__(self, ssd, inp, dev, path, stream):
+        import torch
+        self.ssd, self.inp, self.path, self.stream = ssd, inp, path, stream
+        self.host, self.d = _device_inputs(inp, dev)
+        x = self.d["x"]
+        nseq = inp["workload"].nseq
+        H, P, N = x.shape[2], x.shape[3], self.d["B"].shape[3]
+        self.y = torch.empty_like(x)
+        self.fin = (torch.empty((nseq, H, P, N), dtype=torch.float32, device=dev)
+                    if inp["want_final_states"] else None)
+        self.params = ssd.params_for(x, self.d["B"], inp["chunk_len"], self.d["cu_seqlens"], True, path)
+        self.ws = torch.empty(ssd.workspace_size(self.params), dtype=torch.uint8, device=dev)
+        self.launches = ssd.launch_count(self.params)
+        self.resolved = ssd.resolved_path(self.params)
+
+    def step(self, events=None):
+        d = self.d
+        self.ssd.ssd_fwd(d["x"], d["dt"], d["A_log"], d["B"], d["C"], d["D"], chunk_len=self.inp["chunk_len"],
+                         initial_states=d["initial_states"], cu_seqlens=d["cu_seqlens"], y=self.y,
+                         final_states=self.fin, workspace=self.ws, stream=self.stream, path=self.path,
+                         instrumentation=None if events is None else self.ssd.make_instrumentation(events))
+
+    def status(self):
+        return self.ssd.library().ssd_get_status(self.ws.data_ptr(), self.stream.cuda_stream or None)
+
+    def timed(self, steps, warmup, flush, on_timed_start=None):
+        """Warm-up, then `steps` timed steps (L2 flushed before each); returns
+        per-step lists of (step ms, compute ms, output-pass ms)."""
+        import torch
+        for _ in range(warmup):
+            flush.zero_()
+            self.step()
+        torch.cuda.synchronize()
+        rc = self.status()
+        if rc != 0:
+            raise self.ssd.SsdError(rc, "warm-up device status")
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+        for row in ev:              # torch creates events lazily: record once so the handles exist
+            for e in row:
+                e.record(self.stream)
+        torch.cuda.synchronize()
+        if on_timed_start:
+            on_timed_start()
+        torch.cuda.synchronize()
+        wall0 = time.perf_counter()
+        for i in range(steps):
+            flush.zero_()
+            ev[i][0].record(self.stream)
+            self.step(events=(ev[i][1], ev[i][2], ev[i][3]))
+            ev[i][4].record(self.stream)
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - wall0
+        step_ms = [ev[i][0].elapsed_time(ev[i][4]) for i in range(steps)]
+        comp_ms = [ev[i][1].elapsed_time(ev[i][3]) for i in range(steps)]
+        main_ms = [ev[i][2].elapsed_time(ev[i][3]) for i in range(steps)]
+        return step_ms, comp_ms, main_ms, wall
+
+    def check(self, pairs_wanted=4, seed=1):
+        """Output of the last call against the oracle on sampled (sequence,
+        head) pairs: max|dy| / max|y_oracle| and the same for final states."""
+        import torch
+        import oracle
+        torch.cuda.synchronize()
+        inp = self.inp
+        bounds = ssd_inputs.seq_bounds(inp)
+        H, P = inp["x"].shape[2], inp["x"].shape[3]
+        rng = np.random.default_rng(seed)
+        cand = [(s, h) for s in range(len(bounds)) for h in range(H) if bounds[s][1] > 0]
+        pick = [cand[i] for i in rng.choice(len(cand), size=min(pairs_wanted, len(cand)), replace=False)]
+        ys, fs = oracle.recurrence_pairs(inp, pick)
+        yg = self.y.float().cpu().numpy().reshape(-1, H, P)
+        fg = None if self.fin is None else self.fin.cpu().numpy()
+        ey = ef = 0.0
+        for (s, h), yr, fr in zip(pick, ys, fs):
+            t0, n = bounds[s]
+            ey = max(ey, float(np.max(np.abs(yg[t0:t0 + n, h] - yr)) / max(np.max(np.abs(yr)), 1e-30)))
+            if fg is not None:
+                ef = max(ef, float(np.max(np.abs(fg[s, h] - fr)) / max(np.max(np.abs(fr)), 1e-30)))
+        tol = 2e-2 if inp["io_dtype"] == "bf16" else 1e-4
+        return {"pairs": [list(p) for p in pick], "max_rel_err_y": ey,
+                "max_rel_err_final": ef if fg is not None else None, "tol": tol,
+                "ok": bool(ey <= tol and ef <= tol)}
+
+    def roofline(self, comp_ms, main_ms, workload_name):
+        inp = self.inp
+        alg_bytes = algorithmic_bytes(inp)
+        peak, peak_kind = measured_peaks()
+        kernel = "ssd_tc_walk" if self.resolved == "tensor" else "chunk_scan_kernel"
+        cm = statistics.median(comp_ms)
+        mm = statistics.median(main_ms)
+        achieved = alg_bytes / (cm * 1e-3) / 1e9
+        return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": committed_traffic(workload_name, kernel), "kernel": kernel,
+                "kernel_ms": cm, "alg_bytes": alg_bytes,
+                "timed": "every compute kernel of one forward (CUDA events on the call's stream, median)",
+                "output_pass_ms": mm, "output_pass_frac": alg_bytes / (mm * 1e-3) / 1e9 / peak,
+                "peak_source": f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"}
+
+
+# bf16 workloads measured after the headline (one sub-object each in the JSON line)
+SUB_WORKLOADS = ("small_bf16", "mamba2_2p7b", "long16k_gva", "varlen32k")
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -279,80 +404,42 @@ def run_ours(args):
     torch.cuda.set_device(dev)
 
     inp = make_workload(args)
-    io = torch.bfloat16 if inp["io_dtype"] == "bf16" else torch.float32
-    host = {k: torch.from_numpy(inp[k]).to(io).pin_memory() for k in ("x", "dt", "B", "C")}
-    for k in ("A_log", "D", "initial_states"):
-        host[k] = None if inp[k] is None else torch.from_numpy(inp[k]).pin_memory()
-    host["cu_seqlens"] = None if inp["cu_seqlens"] is None else torch.from_numpy(inp["cu_seqlens"]).pin_memory()
-    d = {k: (None if v is None else v.to(dev)) for k, v in host.items()}
-    x = d["x"]
-    want_final = bool(inp["want_final_states"])
-    nseq = inp["workload"].nseq
-    H, P, N = x.shape[2], x.shape[3], d["B"].shape[3]
-    y = torch.empty_like(x)
-    fin = torch.empty((nseq, H, P, N), dtype=torch.float32, device=dev) if want_final else None
-    params = ssd.params_for(x, d["B"], inp["chunk_len"], d["cu_seqlens"], True, args.path)
-    ws = torch.empty(ssd.workspace_size(params), dtype=torch.uint8, device=dev)
-    launches_per_step = ssd.launch_count(params)
-    path = ssd.resolved_path(params)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
-
-    def step(prof=None):
-        ssd.ssd_fwd(d["x"], d["dt"], d["A_log"], d["B"], d["C"], d["D"], chunk_len=inp["chunk_len"],
-                    initial_states=d["initial_states"], cu_seqlens=d["cu_seqlens"], y=y,
-                    final_states=fin, workspace=ws, stream=stream, path=args.path, prof_events=prof)
-
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
-    torch.cuda.synchronize()
-    rc = ssd.library().ssd_get_status(ws.data_ptr(), stream.cuda_stream or None)
-    if rc != 0:
-        raise ssd.SsdError(rc, "warm-up device status")
+    fw = Forward(ssd, inp, dev, args.path, stream)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
-    for row in ev:              # torch creates events lazily: record once so the handles exist
-        for e in row:
-            e.record(stream)
-    torch.cuda.synchronize()
     sampler = ClockSampler(torch.cuda.current_device() if world == 1 else local)
-    if rank == 0:
-        sampler.start()
-        time.sleep(0.3)
+
+    def start_clocks():
+        if rank == 0:
+            sampler.start()
+            time.sleep(0.3)
+        if world > 1:
+            dist.barrier()
+
+    step_ms, comp_ms, main_ms, wall = fw.timed(K, args.warmup, flush, on_timed_start=start_clocks)
     if world > 1:
         dist.barrier()
-    torch.cuda.synchronize()
-    wall0 = time.perf_counter()
-    for i in range(K):
-        flush.zero_()
-        ev[i][0].record(stream)
-        step(prof=(ev[i][1], ev[i][2]))
-        ev[i][3].record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    wall = time.perf_counter() - wall0
     clocks = sampler.stop() if rank == 0 else None
-    step_ms = [ev[i][0].elapsed_time(ev[i][3]) for i in range(K)]
-    main_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
-    ms, kms = max_over_ranks([statistics.mean(step_ms), statistics.mean(main_ms)], dev)
+    ms, cms = max_over_ranks([statistics.mean(step_ms), statistics.median(comp_ms)], dev)
+    check = fw.check() if rank == 0 else None
 
     # end to end: pinned host inputs -> device -> ssd_fwd -> result back to pinned host memory
+    host, d, y, fin = fw.host, fw.d, fw.y, fw.fin
     y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
     fin_host = torch.empty(fin.shape, dtype=fin.dtype).pin_memory() if fin is not None else None
     h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
     d2h = y_host.numel() * y_host.element_size() + (fin_host.numel() * 4 if fin_host is not None else 0)
     e2e_ms = []
-    for i in range(args.warmup + K):
+    for i in range(args.warmup + min(K, 20)):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         flush.zero_()
         e0.record(stream)
         for k, v in host.items():
             if v is not None:
                 d[k].copy_(v, non_blocking=True)
-        step()
+        fw.step()
         y_host.copy_(y, non_blocking=True)
         if fin_host is not None:
             fin_host.copy_(fin, non_blocking=True)
@@ -363,14 +450,42 @@ def run_ours(args):
     e2e = max_over_ranks([statistics.mean(e2e_ms)], dev)[0]
 
     tokens = inp["x"].shape[0] * inp["x"].shape[1]
-    total_tokens = tokens * world
     value = whole_job_throughput(tokens, world, ms)
-    alg_bytes = algorithmic_bytes(inp)
-    flops = algorithmic_flops(inp)
-    peak, peak_kind = measured_peaks()
-    kernel = "ssd_tc_walk" if path == "tensor" else "chunk_scan_kernel"
-    achieved = alg_bytes / (kms * 1e-3) / 1e9
-    line = None
+    block_len = 128 if fw.resolved == "tensor" else inp["chunk_len"]
+    flops = algorithmic_flops(inp, block_len)
+    roof = fw.roofline(comp_ms, main_ms, args.workload)
+    roof["kernel_ms"] = cms
+    roof["achieved"] = roof["alg_bytes"] / (cms * 1e-3) / 1e9
+    roof["frac"] = roof["achieved"] / roof["peak"]
+
+    # the other workloads, one after another, after the headline's timed region (1 GPU only)
+    subs = {}
+    if args.workload in SUB_WORKLOADS and rank == 0:
+        subs[args.workload] = {"steps": K, "step_ms": _stats(step_ms), "compute_ms": _stats(comp_ms),
+                               "output_pass_ms": _stats(main_ms), "tokens_per_s": tokens / (statistics.median(step_ms) * 1e-3),
+                               "frac": roof["frac"], "output_pass_frac": roof["output_pass_frac"],
+                               "alg_bytes": roof["alg_bytes"], "traffic": roof["traffic"], "path": fw.resolved,
+                               "launches": fw.launches, "check": check, "headline": True}
+    if world == 1 and not args.no_sub_workloads:
+        del fw
+        torch.cuda.empty_cache()
+        for name in SUB_WORKLOADS:
+            if name == args.workload:
+                continue
+            sinp = ssd_inputs.make_inputs(ssd_inputs.workload(name), seed=args.seed)
+            sfw = Forward(ssd, sinp, dev, "auto", stream)
+            sk = max(10, min(K, 50))
+            s_step, s_comp, s_main, _ = sfw.timed(sk, 3, flush)
+            r = sfw.roofline(s_comp, s_main, name)
+            stoks = sinp["x"].shape[0] * sinp["x"].shape[1]
+            subs[name] = {"steps": sk, "step_ms": _stats(s_step), "compute_ms": _stats(s_comp),
+                          "output_pass_ms": _stats(s_main), "tokens_per_s": stoks / (statistics.median(s_step) * 1e-3),
+                          "frac": r["frac"], "output_pass_frac": r["output_pass_frac"], "alg_bytes": r["alg_bytes"],
+                          "traffic": r["traffic"], "path": sfw.resolved, "launches": sfw.launches,
+                          "check": sfw.check()}
+            del sfw
+            torch.cuda.empty_cache()
+
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
@@ -382,24 +497,33 @@ def run_ours(args):
             "scaling": "weak", "vs_baseline": None, "dtype": inp["io_dtype"],
             "data": "synthetic (seeded generator, value distributions of the workload)",
             "config": config_of(inp, args, world),
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": committed_traffic(args.workload, kernel),
-                         "kernel": kernel, "kernel_ms": kms, "alg_bytes": alg_bytes,
-                         "peak_source": f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"},
-            "tflops": flops / (ms * 1e-3) / 1e12,
+            "step_ms": _stats(step_ms), "compute_ms": _stats(comp_ms), "output_pass_ms": _stats(main_ms),
+            "roofline": roof,
+            "tflops": flops / (ms * 1e-3) / 1e12, "flops_block_len": block_len,
+            "check": check,
             "cpu_baseline": cpu,
             "e2e": {"value": whole_job_throughput(tokens, world, e2e), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": launches_per_step * K,
+            "gpu_launches": fw_launches(ssd, inp, args.path) * K,
             "clocks": clocks,
-            "path": path,
+            "path": ssd.resolved_path(ssd.params_for(d["x"], d["B"], inp["chunk_len"], d["cu_seqlens"], True,
+                                                     args.path)),
             "wall_s_timed_region": wall,
+            "workloads": subs,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def fw_launches(ssd, inp, path):
+    w = inp["workload"]
+    p = ssd.make_params(batch=w.batch, seqlen=w.seqlen, nheads=w.nheads, headdim=w.headdim, dstate=w.dstate,
+                        ngroups=w.ngroups, chunk_len=inp["chunk_len"], num_seqs=w.num_seqs, io_dtype=w.io_dtype,
+                        path=path)
+    return ssd.launch_count(p)
 
 
 DECODE_METRIC = "SSD decode step tokens/s at 1 B200; % of HBM roofline"
@@ -539,14 +663,16 @@ def run_decode(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mamba2_2p7b", choices=sorted(ssd_inputs.WORKLOADS))
     ap.add_argument("--path", default="auto", choices=["auto", "simt", "tensor"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--ref-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sub-workloads", action="store_true",
+                    help="skip the per-workload measurements that follow the headline")
     ap.add_argument("--op", choices=["fwd", "decode"], default="fwd",
                     help="fwd: the chunked forward (default); decode: one recurrent step per row")
     args = ap.parse_args()

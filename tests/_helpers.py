@@ -7,6 +7,14 @@ import ssd_inputs
 BF16_TOL = 2e-2   # max|dy| / max|y_oracle| for bf16 inputs
 F32_TOL = 1e-4    # same, float32 path
 
+# (test, y error, final-state error, tolerance) of the parity checks that ran,
+# printed in pytest's terminal summary so that every margin is on record
+PARITY_LOG = []
+
+
+def record_parity(name, ey, ef, tol):
+    PARITY_LOG.append((name, float(ey), None if ef is None else float(ef), float(tol)))
+
 
 def to_device(inp: dict, device="cuda"):
     import torch
