@@ -140,8 +140,21 @@ constexpr size_t tc_smem_bytes()
 
 __device__ __forceinline__ void record_timeout(int *status) { set_status(status, kDevTimeout); }
 
-// TMEM column map
-constexpr uint32_t kColCB = 0, kColPm = 128, kColH = 256, kColYd = 384, kColYo = 448;
+// TMEM column map (512 columns): CB at 0, the Pm buffers from 128, every
+// head's state from 256.  With two heads at dstate 256 the states fill
+// 256..511, so Pm is single-buffered and Yd and Yo share one accumulator at
+// 192 (the epilogue reads Yo before Pm X overwrites it); otherwise Pm is
+// double-buffered and Yd, Yo sit at 384 and 448.
+constexpr uint32_t kColCB = 0, kColPm = 128, kColH = 256;
+template <int NST, int KH>
+struct TmemMap {
+    static constexpr int kMT = NST >= 256 ? 2 : 1;                 // 128-row state tiles per head
+    static constexpr bool kSharedY = KH * kMT * 64 > 128;
+    static constexpr int kPmBufs = kSharedY ? 1 : 2;
+    static constexpr uint32_t kColYd = kSharedY ? 192u : 384u;
+    static constexpr uint32_t kColYo = kSharedY ? 192u : 448u;
+    static_assert(kColH + KH * kMT * 64 <= 512, "states do not fit in tensor memory");
+};
 
 // Optional per-CTA event timeline (SM clock), compiled only with -DSSD_TRACE.
 #ifdef SSD_TRACE
@@ -206,7 +219,31 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
     // dstate 256 (one head per item): C bf16(H)^T is issued by the state issuer, so it
     // never queues behind the mask-bound Pm X (+3 % there; slower with two heads)
     constexpr bool kYoOnState = !STATE_ONLY && NST >= 256;
-    constexpr int kMT = NST >= 256 ? 2 : 1;        // 128-row state tiles per head (H^T rows = n)
+    constexpr int kMT = TmemMap<NST, KH>::kMT;     // 128-row state tiles per head (H^T rows = n)
+    constexpr bool kSharedY = !STATE_ONLY && TmemMap<NST, KH>::kSharedY;
+    constexpr int kPmB = TmemMap<NST, KH>::kPmBufs;
+    constexpr uint32_t kColYd = TmemMap<NST, KH>::kColYd, kColYo = TmemMap<NST, KH>::kColYo;
+    // the shared Y accumulator needs Yo issued by the state issuer (its own yo_full commit)
+    static_assert(!kSharedY || kYoOnState, "shared Yd/Yo accumulator needs the state issuer to issue Yo");
+    // state-only mode at dstate 256 runs a two-stage B ring in the C and B slots of the single B/C stage
+    constexpr int kBR = (STATE_ONLY && kSt == 1) ? 2 : kSt;
+    // one B/C stage with outputs: B and C have their own full/empty barriers (C: bc_*[0], B: bc_*[1]),
+    // so the next block's B loads once the last state UMMA is done, while C still feeds C Hbf^T
+    constexpr bool kSplitBC = !STATE_ONLY && kSt == 1;
+    static_assert(!kSplitBC || kYoOnState, "a split B/C stage assumes the state issuer issues C Hbf^T");
+    // two heads sharing Yd/Yo: the second head's Pm is written over the CB columns its mask has
+    // just read (K steps 0-3 at columns 0-31, 4-7 at 64-95), so it does not wait for the first
+    // head's Pm X; the next CB waits for that Pm X instead
+    constexpr bool kInPlace = kSharedY && KH == 2;
+    // state-only mode: one state UMMA per block for both heads (N = 128, the B^T operand read once);
+    // the heads' states are adjacent per 128-row tile (column kColH + 64 (j + KH mt)) and so are
+    // their w o X tiles (at dstate 256 in the bf16(H) tile, which state-only mode does not use)
+    constexpr bool kMergeSt = STATE_ONLY && KH == 2;
+    constexpr int kXwR = (STATE_ONLY && kXwD == 1) ? 2 : kXwD;     // w o X ring depth
+    auto xw_tile = [&](int i) -> uint8_t * { return (STATE_ONLY && kXwD == 1) ? S.hbf + 16384 * i : S.xw[i]; };
+    auto b_tile = [&](int stage) -> uint8_t * {
+        return (STATE_ONLY && kSt == 1) ? S.bc[0][stage][0] : S.bc[stage][1][0];
+    };
 
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
@@ -248,7 +285,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
     const uint32_t tb = S.tmem_base;
 #ifdef SSD_TRACE
     const long long t_start = clock64();
-    long long *const trace_buf = blockIdx.x < kTraceCtas ? g_trace : nullptr;
+    long long *const trace_buf = (blockIdx.x < kTraceCtas && !STATE_ONLY) ? g_trace : nullptr;
 #endif
 
     if (warp == 0) {
@@ -258,9 +295,14 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
         float Areg[KH];
 #pragma unroll
         for (int j = 0; j < KH; ++j) Areg[j] = -expf(prm.A_log[it.h0 + j]);
+        // state-only mode walks the segment backwards: rsum[j] = log decay of the blocks
+        // already walked (those after the current one), folded into w
+        float rsum[KH];
+#pragma unroll
+        for (int j = 0; j < KH; ++j) rsum[j] = 0.0f;
         bool ok = true;
         for (int u = 0; u < nunits && ok; ++u) {
-            const int c = u / KH, j = u % KH, slot = u % kCsd;
+            const int c = STATE_ONLY ? nblk - 1 - u / KH : u / KH, j = u % KH, slot = u % kCsd;
             const int row0 = it.tok0 + c * kQ;
             const int valid = min(kQ, it.len - c * kQ);
             const int h = it.h0 + j;
@@ -296,12 +338,22 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             }
             const float excl = incl - run;
             const float last = __shfl_sync(0xffffffffu, incl, 31);
+            float rs = 0.0f;
+            if (STATE_ONLY) {
+#pragma unroll
+                for (int jj = 0; jj < KH; ++jj)
+                    if (j == jj) {
+                        rs = rsum[jj];
+                        rsum[jj] += last;
+                    }
+            }
             float c2v[4], wv[4], ev[4], uv[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const float csn = excl + pre[i];
                 c2v[i] = csn * kLog2e;
-                wv[i] = ex2_approx((last - csn) * kLog2e) * dl[i];
+                // decay from token s to the block end (and, walking backwards, on to the segment end)
+                wv[i] = ex2_approx((STATE_ONLY ? last - csn + rs : last - csn) * kLog2e) * dl[i];
                 ev[i] = ex2_approx(c2v[i]);
             }
             // factorised mask: exp2(cs2_l - cs2_s) = exp2(cs2_l - R) * exp2(R - cs2_s) with R the
@@ -332,35 +384,68 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             const bool leader = elect_one();
             const uint32_t id_h = idesc_bf16_f32(128, kP, true, true);
             const uint32_t id_y = idesc_bf16_f32(128, kP, false, true);
+            const uint32_t id_h2 = idesc_bf16_f32(128, 2 * kP, true, true);
             const uint32_t lbo_m = NST >= 128 ? 16384u : 0u;   // N = 64: rows 64..127 repeat rows 0..63
             bool ok = true;
             for (int c = 0; c < nblk && ok; ++c) {
-                const int bs = c % kSt;
-                ok = mbar_wait<kInlW>(&S.bc_full[bs], (c / kSt) & 1, abort);
+                const int bs = c % kBR;
+                ok = mbar_wait<kInlW>(&S.bc_full[kSplitBC ? 1 : bs], (c / kBR) & 1, abort);
                 if (!ok) break;
-                const uint32_t sB = smem_u32(S.bc[bs][1][0]);
-                for (int j = 0; j < KH && ok; ++j) {
-                    const int u = c * KH + j, wi = u % kXwD;
-                    ok = mbar_wait<kInlW>(&S.xw_full[wi], (u / kXwD) & 1, abort) && mbar_wait<kInlW>(&S.hs_full[j], c & 1, abort);
-                    SSD_TRACE_EV(15, u);
+                const uint32_t sB = smem_u32(b_tile(bs));
+                if (kMergeSt) {
+                    // both heads: w o X tiles 0 and 1 (u = 2c, 2c + 1) form one N = 128 operand
+                    ok = mbar_wait<kInlW>(&S.xw_full[0], c & 1, abort) && mbar_wait<kInlW>(&S.xw_full[1], c & 1, abort) &&
+                         (c > 0 || (mbar_wait<kInlW>(&S.hs_full[0], 0, abort) && mbar_wait<kInlW>(&S.hs_full[1], 0, abort)));
                     if (!ok) break;
                     tc_fence_after();
-                    const uint64_t b0 = sdesc_sw128(smem_u32(S.xw[wi]), 16384, 1024);
+                    const uint64_t b0 = sdesc_sw128(smem_u32(xw_tile(0)), 16384, 1024);
 #pragma unroll
                     for (int mt = 0; mt < kMT; ++mt) {
                         const uint64_t a0 = sdesc_sw128(sB + mt * 32768, lbo_m, 1024);
 #pragma unroll
                         for (int kk = 0; kk < kQ / 16; ++kk)
                             if (leader)
-                                umma_ss(tb + kColH + 64 * (j * kMT + mt), desc_adv(a0, kk * 2048),
+                                umma_ss(tb + kColH + 64 * KH * mt, desc_adv(a0, kk * 2048), desc_adv(b0, kk * 2048),
+                                        id_h2, 1);
+                    }
+                    if (leader) {
+                        umma_commit(&S.xw_empty[0]);
+                        umma_commit(&S.xw_empty[1]);
+                        umma_commit(&S.h_ready[0]);
+                        umma_commit(&S.h_ready[1]);
+                        umma_commit(&S.bc_empty[bs]);
+                    }
+                    continue;
+                }
+                for (int j = 0; j < KH && ok; ++j) {
+                    const int u = c * KH + j, wi = u % kXwR;
+                    // state-only mode never rescales: hs_full[j] completes once, when the zeroed state is in place
+                    ok = mbar_wait<kInlW>(&S.xw_full[wi], (u / kXwR) & 1, abort) &&
+                         (STATE_ONLY ? (c > 0 || mbar_wait<kInlW>(&S.hs_full[j], 0, abort))
+                                     : mbar_wait<kInlW>(&S.hs_full[j], c & 1, abort));
+                    SSD_TRACE_EV(15, u);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint64_t b0 = sdesc_sw128(smem_u32(xw_tile(wi)), 16384, 1024);
+#pragma unroll
+                    for (int mt = 0; mt < kMT; ++mt) {
+                        const uint64_t a0 = sdesc_sw128(sB + mt * 32768, lbo_m, 1024);
+#pragma unroll
+                        for (int kk = 0; kk < kQ / 16; ++kk)
+                            if (leader)
+                                umma_ss(tb + kColH + 64 * (j + KH * mt), desc_adv(a0, kk * 2048),
                                         desc_adv(b0, kk * 2048), id_h, 1);
                     }
                     if (leader) umma_commit(kTmaY ? &S.xw_free[wi] : &S.xw_empty[wi]);
                     if (leader) umma_commit(&S.h_ready[j]);
+                    if (kSplitBC && j == KH - 1 && leader) umma_commit(&S.bc_empty[1]);   // B of block c done
                     SSD_TRACE_EV(4, u);
                     if (kYoOnState) {
+                        // the accumulator is free once the epilogue has read the previous unit's
+                        // Yo (its own columns) or Yd (columns shared with Yo)
                         ok = mbar_wait<kInlW>(&S.hb_full, u & 1, abort) &&
-                             (u == 0 || mbar_wait<kInlW>(&S.yo_empty, (u - 1) & 1, abort));
+                             (u == 0 || mbar_wait<kInlW>(kSharedY ? &S.yd_empty : &S.yo_empty, (u - 1) & 1, abort)) &&
+                             (!kSplitBC || j > 0 || mbar_wait<kInlW>(&S.bc_full[0], c & 1, abort));
                         if (!ok) break;
                         tc_fence_after();
                         const uint64_t c0 = sdesc_sw128(smem_u32(S.bc[bs][0][0]), 16, 1024);
@@ -373,9 +458,10 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                         }
                         if (leader) umma_commit(&S.hb_empty);
                         if (leader) umma_commit(&S.yo_full);
+                        SSD_TRACE_EV(27, u);
                     }
                 }
-                if (leader) umma_commit(&S.bc_empty[bs]);
+                if (leader) umma_commit(&S.bc_empty[kSplitBC ? 0 : bs]);   // (C of block c done)
             }
             if (leader) umma_commit(&S.drain_s);
             mbar_wait<kInlW>(&S.drain_s, 0, abort, 200000000ull);
@@ -390,45 +476,74 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             constexpr uint32_t kBcBytes = (STATE_ONLY ? 1 : 2) * (NST / 64) * kBoxBytes;
             int issued_bc[2] = {-1, -1}, issued_x[2] = {-1, -1};
             bool ok = true;
-            // L2 prefetch runs kPrefetch blocks ahead of the shared-memory ring
+            // L2 prefetch runs kPF blocks ahead of the shared-memory ring
+            constexpr int kPF = STATE_ONLY ? 1 : (NST >= 256 ? 2 : kPrefetch);
             auto prefetch = [&](int c) {
-                const int row = it.tok0 + c * kQ;
+                const int row = it.tok0 + (STATE_ONLY ? nblk - 1 - c : c) * kQ;   // state-only: backwards
                 for (int b = 0; b < NST / 64; ++b) {
                     if (!STATE_ONLY) tma_prefetch_l2_2d(&mapC, g * NST + 64 * b, row);
                     tma_prefetch_l2_2d(&mapB, g * NST + 64 * b, row);
                 }
                 for (int j = 0; j < KH; ++j) tma_prefetch_l2_2d(&mapX, (it.h0 + j) * kP, row);
             };
-            for (int c = 0; c < nblk && ok; ++c) {
-                const int bs = c % kSt;
-#pragma unroll 1
-                for (int pc = c == 0 ? 0 : c + kPrefetch; pc <= c + kPrefetch && pc < nblk; ++pc) prefetch(pc);
-                if (c >= kSt) ok = mbar_wait<kInlW>(&S.bc_empty[bs], ((c / kSt) + 1) & 1, abort);
-                if (!ok) break;
-                const int row = it.tok0 + c * kQ;
+            // split B/C stage: one half (1 = B, 0 = C) of block c
+            auto load_half = [&](int c, int half) -> bool {
+                const int row = it.tok0 + (STATE_ONLY ? nblk - 1 - c : c) * kQ;   // state-only: backwards
+                if (c >= 1 && !mbar_wait<kInlW>(&S.bc_empty[half], (c + 1) & 1, abort)) return false;
+                mbar_arrive_expect_tx(&S.bc_full[half], (NST / 64) * 16384u);
+                for (int b = 0; b < NST / 64; ++b)
+                    tma_load_2d(S.bc[0][half][b], half ? &mapB : &mapC, &S.bc_full[half], g * NST + 64 * b, row);
+                issued_bc[half] = c;
+                if (half == 0) SSD_TRACE_EV(0, c);
+                return true;
+            };
+            auto load_bc = [&](int c) -> bool {
+                const int row = it.tok0 + (STATE_ONLY ? nblk - 1 - c : c) * kQ;   // state-only: backwards
+                const int bs = c % kBR;
+                if (c >= kBR && !mbar_wait<kInlW>(&S.bc_empty[bs], ((c / kBR) + 1) & 1, abort)) return false;
                 mbar_arrive_expect_tx(&S.bc_full[bs], kBcBytes);
+                uint8_t *bdst = b_tile(bs);
                 for (int b = 0; b < NST / 64; ++b) {
                     if (!STATE_ONLY) tma_load_2d(S.bc[bs][0][b], &mapC, &S.bc_full[bs], g * NST + 64 * b, row);
-                    tma_load_2d(S.bc[bs][1][b], &mapB, &S.bc_full[bs], g * NST + 64 * b, row);
+                    tma_load_2d(bdst + 16384 * b, &mapB, &S.bc_full[bs], g * NST + 64 * b, row);
                 }
                 issued_bc[bs] = c;
                 SSD_TRACE_EV(0, c);
-                for (int j = 0; j < KH; ++j) {
+                return true;
+            };
+            auto load_x = [&](int c, int j0, int j1) -> bool {
+                const int row = it.tok0 + (STATE_ONLY ? nblk - 1 - c : c) * kQ;   // state-only: backwards
+                for (int j = j0; j < j1; ++j) {
                     const int u = c * KH + j, xs = u & 1;
-                    if (u >= 2) ok = mbar_wait<kInlW>(&S.x_empty[xs], ((u >> 1) + 1) & 1, abort);
-                    if (!ok) break;
+                    if (u >= 2 && !mbar_wait<kInlW>(&S.x_empty[xs], ((u >> 1) + 1) & 1, abort)) return false;
                     if (prm.withhold_x0 && item_idx == 0 && u == 0) continue;
                     mbar_arrive_expect_tx(&S.x_full[xs], kBoxBytes);
                     tma_load_2d(S.x[xs], &mapX, &S.x_full[xs], (it.h0 + j) * kP, row);
                     issued_x[xs] = u;
                     SSD_TRACE_EV(1, u);
                 }
+                return true;
+            };
+            for (int c = 0; c < nblk && ok; ++c) {
+#pragma unroll 1
+                for (int pc = c == 0 ? 0 : c + kPF; pc <= c + kPF && pc < nblk; ++pc) prefetch(pc);
+                // the single-threaded producer requests tiles in the order their slots free up:
+                // with a split B/C stage B (last state UMMA), x of the first heads (their Pm X),
+                // C (last C Hbf^T), x of the last head (the block's final Pm X)
+                if (kSplitBC)
+                    ok = load_half(c, 1) && load_x(c, 0, KH - 1) && load_half(c, 0) && load_x(c, KH - 1, KH);
+                else if (kBR == 1)
+                    ok = load_x(c, 0, KH) && load_bc(c);
+                else
+                    ok = load_bc(c) && load_x(c, 0, KH);
             }
             if (!ok) {
                 // drain: wait (bounded) for copies still in flight before the CTA exits
                 for (int i = 0; i < 2; ++i) {
-                    if (i < kSt && issued_bc[i] >= 0)
-                        mbar_wait<kInlW>(&S.bc_full[i], (issued_bc[i] / kSt) & 1, abort, 200000000ull);
+                    if (kSplitBC && issued_bc[i] >= 0)
+                        mbar_wait<kInlW>(&S.bc_full[i], issued_bc[i] & 1, abort, 200000000ull);
+                    else if (i < kBR && issued_bc[i] >= 0)
+                        mbar_wait<kInlW>(&S.bc_full[i], (issued_bc[i] / kBR) & 1, abort, 200000000ull);
                     if (issued_x[i] >= 0) mbar_wait<kInlW>(&S.x_full[i], (issued_x[i] >> 1) & 1, abort, 200000000ull);
                 }
             }
@@ -445,7 +560,10 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             auto issue_cb = [&](int c) -> bool {
                 const int bs = c % kSt;
                 if (!mbar_wait<kInlW>(&S.bc_full[bs], (c / kSt) & 1, abort)) return false;
+                if (kSplitBC && !mbar_wait<kInlW>(&S.bc_full[1], c & 1, abort)) return false;
                 if (c >= 1 && !mbar_wait<kInlW>(&S.cb_empty, (c - 1) & 1, abort)) return false;
+                // the previous block's last Pm lives in the CB columns until its Pm X is done
+                if (kInPlace && c >= 1 && !mbar_wait<kInlW>(&S.pm_empty[1], (c - 1) & 1, abort)) return false;
                 tc_fence_after();
                 const uint64_t a0 = sdesc_sw128(smem_u32(S.bc[bs][0][0]), 16, 1024);
                 const uint64_t b0 = sdesc_sw128(smem_u32(S.bc[bs][1][0]), 16, 1024);
@@ -455,6 +573,11 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                     if (leader) umma_ss(tb + kColCB, desc_adv(a0, off), desc_adv(b0, off), id_cb, kk > 0);
                 }
                 if (leader) umma_commit(&S.cb_full);
+                if (kYoOnState && leader) {
+                    // CB is this issuer's only use of B and C
+                    umma_commit(&S.bc_empty[0]);
+                    if (kSplitBC) umma_commit(&S.bc_empty[1]);
+                }
                 SSD_TRACE_EV(2, c);
                 return true;
             };
@@ -469,7 +592,10 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                     if (!ok) break;
                 }
                 for (int j = 0; j < KH && ok; ++j) {
-                    const int u = c * KH + j, xs = u & 1, pi = u & 1;
+                    const int u = c * KH + j, xs = u & 1;
+                    // Pm buffer (barrier index) of this unit and the phase it completes
+                    const int pi = kInPlace ? j : u % kPmB;
+                    const int pph = kInPlace ? (c & 1) : ((u / kPmB) & 1);
                     // Yo = C Hbf^T (issued by the state issuer when kYoOnState)
                     if (!kYoOnState) {
                         ok = mbar_wait<kInlW>(&S.hb_full, u & 1, abort);
@@ -492,24 +618,29 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                         ok = issue_cb(c + 1);
                         if (!ok) break;
                     }
-                    // Yd = Pm X
-                    ok = mbar_wait<kInlW>(&S.pm_full[pi], (u >> 1) & 1, abort) &&
+                    // Yd = Pm X, once the accumulator is free: the previous Yd read, or (shared
+                    // with Yo) this unit's Yo read
+                    ok = mbar_wait<kInlW>(&S.pm_full[pi], pph, abort) &&
                          mbar_wait<kInlW>(&S.x_full[xs], (u >> 1) & 1, abort) &&
-                         (u == 0 || mbar_wait<kInlW>(&S.yd_empty, (u - 1) & 1, abort));
+                         (kSharedY ? mbar_wait<kInlW>(&S.yo_empty, u & 1, abort)
+                                   : (u == 0 || mbar_wait<kInlW>(&S.yd_empty, (u - 1) & 1, abort)));
                     SSD_TRACE_EV(16, u);
                     if (!ok) break;
                     tc_fence_after();
                     const uint64_t x0 = sdesc_sw128(smem_u32(S.x[xs]), 16384, 1024);
-                    const uint32_t pm = tb + kColPm + 64 * pi;
+                    const bool ip = kInPlace && j == 1;
+                    const uint32_t pm = ip ? tb + kColCB : tb + kColPm + 64 * pi;
 #pragma unroll
-                    for (int kk = 0; kk < kQ / 16; ++kk)
-                        if (leader) umma_ts(tb + kColYd, pm + kk * 8, desc_adv(x0, kk * 2048), id_y, kk > 0);
+                    for (int kk = 0; kk < kQ / 16; ++kk) {
+                        const uint32_t acol = pm + kk * 8 + (ip && kk >= 4 ? 32u : 0u);
+                        if (leader) umma_ts(tb + kColYd, acol, desc_adv(x0, kk * 2048), id_y, kk > 0);
+                    }
                     if (leader) umma_commit(&S.pm_empty[pi]);
                     if (leader) umma_commit(&S.y_full);
                     if (leader) umma_commit(&S.x_empty[xs]);
                     SSD_TRACE_EV(5, u);
                 }
-                if (leader) umma_commit(&S.bc_empty[bs]);
+                if (!kYoOnState && leader) umma_commit(&S.bc_empty[bs]);
             }
             // every UMMA issued so far has completed before TMEM is released
             if (leader) umma_commit(&S.drain_o);
@@ -536,9 +667,14 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                 if (!ok) break;
                 tc_fence_after();
                 for (int j = 0; j < KH; ++j) {
-                    const int u = c * KH + j, slot = u % kCsd, pi = u & 1;
-                    ok = mbar_wait<kInlW>(&S.cs_full[slot], (u / kCsd) & 1, abort) &&
-                         (u < 2 || mbar_wait<kInlW>(&S.pm_empty[pi], ((u >> 1) + 1) & 1, abort));
+                    const int u = c * KH + j, slot = u % kCsd;
+                    const bool ip = kInPlace && j == 1;    // written over the CB columns just read
+                    const int pi = kInPlace ? j : u % kPmB;
+                    ok = mbar_wait<kInlW>(&S.cs_full[slot], (u / kCsd) & 1, abort);
+                    if (kInPlace)
+                        ok = ok && (ip || c == 0 || mbar_wait<kInlW>(&S.pm_empty[0], (c - 1) & 1, abort));
+                    else
+                        ok = ok && (u < kPmB || mbar_wait<kInlW>(&S.pm_empty[pi], ((u / kPmB) + 1) & 1, abort));
                     if (!ok) break;
                     tc_fence_after();
                     if (warp == 4 && lane == 0) SSD_TRACE_EV(7, u);
@@ -548,7 +684,8 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
 #pragma unroll
                     for (int jj = 1; jj < KH; ++jj)
                         if (j == jj) Dh = Dreg[jj];
-                    const uint32_t pm_col = tb + lane_base + kColPm + 64 * pi + half * 32;
+                    const uint32_t pm_col =
+                        ip ? tb + lane_base + kColCB + half * 64 : tb + lane_base + kColPm + 64 * pi + half * 32;
                     const bool exact = S.exact[slot] != 0;
 #pragma unroll 1
                     for (int pair = 0; pair < 2; ++pair) {      // 32 columns -> 16 TMEM columns
@@ -627,6 +764,15 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&S.cb_empty);
                     }
+                    if (ip && q < 2) {
+                        // rows 0..63: K steps 4-7 (columns 64-95 in place) lie above the diagonal; nothing
+                        // else touches these columns of these rows, which the CB UMMA filled
+                        uint32_t zeros[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) zeros[i] = 0u;
+                        tmem_st16(tb + lane_base + kColCB + 64, zeros);
+                        tmem_st16(tb + lane_base + kColCB + 80, zeros);
+                    }
                     tmem_st_wait();
                     tc_fence_before();
                     __syncwarp();
@@ -646,7 +792,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
 #pragma unroll
             for (int i = 0; i < 16; ++i) zeros[i] = 0u;
 #pragma unroll
-            for (int pi = 0; pi < 2; ++pi)
+            for (int pi = 0; pi < kPmB; ++pi)
 #pragma unroll
                 for (int pair = 0; pair < 2; ++pair) tmem_st16(tb + lane_base + kColPm + 64 * pi + 32 + 16 * pair, zeros);
             tmem_st_wait();
@@ -655,10 +801,10 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
         bool ok = true;
         const int r0 = (warp - 8) * 64 + lane;          // rows r0 and r0 + 32
         for (int u = 0; u < nunits && ok; ++u) {
-            const int slot = u % kCsd, xs = u & 1, wi = u % kXwD;
+            const int slot = u % kCsd, xs = u & 1, wi = u % kXwR;
             ok = mbar_wait<kInlW>(&S.cs_full[slot], (u / kCsd) & 1, abort) &&
                  mbar_wait<kInlW>(&S.x_full[xs], (u >> 1) & 1, abort) &&
-                 (u < kXwD || mbar_wait<kInlW>(&S.xw_empty[wi], ((u / kXwD) + 1) & 1, abort));
+                 (u < kXwR || mbar_wait<kInlW>(&S.xw_empty[wi], ((u / kXwR) + 1) & 1, abort));
             if (!ok) break;
             if (warp == 8 && lane == 0) SSD_TRACE_EV(25, u);
             {
@@ -684,7 +830,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                         __nv_bfloat162 *pv = reinterpret_cast<__nv_bfloat162 *>(&v[rr][ch]);
 #pragma unroll
                         for (int i = 0; i < 4; ++i) pv[i] = __hmul2(pv[i], ws2);
-                        *reinterpret_cast<uint4 *>(S.xw[wi] + t * 128 + ((ch * 16) ^ rot)) = v[rr][ch];
+                        *reinterpret_cast<uint4 *>(xw_tile(wi) + t * 128 + ((ch * 16) ^ rot)) = v[rr][ch];
                     }
                 }
             }
@@ -720,7 +866,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                     uint32_t r[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) r[i] = src ? __float_as_uint(src[(size_t)(p0 + i) * N + n]) : 0u;
-                    tmem_st16(tb + lane_base + kColH + 64 * (j * kMT + mt) + p0, r);
+                    tmem_st16(tb + lane_base + kColH + 64 * (j + KH * mt) + p0, r);
                 }
             }
         }
@@ -734,7 +880,8 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
         // epilogue of unit v: y = Yd + exp(cs_l) Yo for this thread's row
         auto epilogue = [&](int v) -> bool {
             const int c = v / KH, j = v % KH, slot = v % kCsd;
-            if (!mbar_wait<kInlW>(&S.y_full, v & 1, abort)) return false;
+            // Yd and Yo in one accumulator: Yo is read first, then Pm X may write Yd
+            if (!kSharedY && !mbar_wait<kInlW>(&S.y_full, v & 1, abort)) return false;
             if (kYoOnState && !mbar_wait<kInlW>(&S.yo_full, v & 1, abort)) return false;
             tc_fence_after();
             if (warp == 12 && lane == 0) SSD_TRACE_EV(12, v);
@@ -751,6 +898,11 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             __syncwarp();
             if (lane == 0) mbar_arrive(&S.yo_empty);
             if (warp == 12 && lane == 0) SSD_TRACE_EV(26, v);
+            if (kSharedY) {
+                if (!mbar_wait<kInlW>(&S.y_full, v & 1, abort)) return false;
+                tc_fence_after();
+                if (warp == 12 && lane == 0) SSD_TRACE_EV(17, v);
+            }
             __nv_bfloat16 *dst = prm.y + ((size_t)tok * prm.H + it.h0 + j) * kP;
             const int wi = v % kXwD;
             uint8_t *stage = S.xw[wi] + q * 32 * 128;     // this warp's 32 rows, 128-byte swizzled
@@ -790,12 +942,14 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             }
             if (via_tma) fence_async_smem();
             __syncwarp();
+            if (warp == 12 && lane == 0) SSD_TRACE_EV(23, v);
             if (lane == 0) {
                 if (via_tma) {
                     tma_store_2d(&mapY, stage, (it.h0 + j) * kP, it.tok0 + c * kQ + q * 32);
                     bulk_commit();
                     bulk_wait_read_all();
                 }
+                if (warp == 12) SSD_TRACE_EV(24, v);
                 if (kTmaY) mbar_arrive(&S.xw_empty[wi]);
                 mbar_arrive(&S.cs_empty[slot]);
             }
@@ -809,6 +963,23 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                 break;
             }
             const int c = u / KH, j = u % KH, slot = u % kCsd;
+            if (STATE_ONLY) {
+                // backward walk: the state is one accumulation from zero, never rescaled
+                if (c == 0) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&S.hs_full[j]);   // the zeroed state is in place
+                }
+                ok = mbar_wait<kInlW>(&S.cs_full[slot], (u / kCsd) & 1, abort);
+                if (!ok) break;
+                const float ld = S.ldec[slot];
+#pragma unroll
+                for (int jj = 0; jj < KH; ++jj)
+                    if (j == jj) ldec_sum[jj] += ld;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.cs_empty[slot]);
+                continue;
+            }
             ok = mbar_wait<kInlW>(&S.cs_full[slot], (u / kCsd) & 1, abort) &&
                  (c == 0 || mbar_wait<kInlW>(&S.h_ready[j], (c - 1) & 1, abort));
             if (!ok) break;
@@ -824,7 +995,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             // H pass: Hbf = bf16(H) (rows n, MN-major), H <- alpha * H in place
 #pragma unroll
             for (int mt = 0; mt < kMT; ++mt) {
-                const uint32_t hcol = tb + lane_base + kColH + 64 * (j * kMT + mt);
+                const uint32_t hcol = tb + lane_base + kColH + 64 * (j + KH * mt);
                 const int n = t + 128 * mt;
                 uint32_t r[64];
 #pragma unroll
@@ -878,7 +1049,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                     dst = prm.final_states + ((size_t)it.seq * prm.H + h) * PN;
 #pragma unroll
                 for (int mt = 0; mt < kMT; ++mt) {
-                    const uint32_t hcol = tb + lane_base + kColH + 64 * (j * kMT + mt);
+                    const uint32_t hcol = tb + lane_base + kColH + 64 * (j + KH * mt);
                     const int n = t + 128 * mt;
 #pragma unroll
                     for (int p0 = 0; p0 < kP; p0 += 16) {
@@ -1128,8 +1299,8 @@ TcPlanShape plan_shape(const ssd_fwd_params &p)
 {
     TcPlanShape s;
     const int hpg = p.nheads / p.ngroups;
-    // two heads per CTA share B/C tiles; dstate 256 leaves TMEM for one head's state
-    s.KH = (hpg % 2 == 0 && p.dstate <= 128) ? 2 : 1;
+    // two heads per CTA share B/C tiles (at dstate 256 with one Yd/Yo accumulator)
+    s.KH = hpg % 2 == 0 ? 2 : 1;
     s.n_hb = p.nheads / s.KH;
     const int nseq = p.num_seqs > 0 ? p.num_seqs : p.batch;
     const long long tokens = (long long)p.batch * p.seqlen;
@@ -1190,7 +1361,7 @@ template <bool SO>
 cudaError_t launch_walk_any(int N, int KH, int grid, const CUtensorMap &mX, const CUtensorMap &mB,
                             const CUtensorMap &mC, const CUtensorMap &mY, const TcParams &prm, cudaStream_t st)
 {
-    if (N == 256) return launch_walk<256, 1, SO>(grid, mX, mB, mC, mY, prm, st);
+    if (N == 256) return launch_walk_kh<256, SO>(KH, grid, mX, mB, mC, mY, prm, st);
     return N == 128 ? launch_walk_kh<128, SO>(KH, grid, mX, mB, mC, mY, prm, st)
                     : launch_walk_kh<64, SO>(KH, grid, mX, mB, mC, mY, prm, st);
 }
