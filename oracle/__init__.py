@@ -11,6 +11,8 @@ Structured State Space Duality":
 * `recurrence` - the linear (recurrent) mode, Sec. 3.4.1 eq. (8): expand by B,
   scalar recurrence, contract by C. Plain C in `ssd_ref.c`, fp64, threads over
   (sequence, head) pairs. This is the oracle the CUDA path is compared with.
+* `recurrence_grad` - reverse mode of the same recurrence (every input's
+  gradient given dL/dy and dL/dfinal), plain C, fp64.
 * `quadratic_form` - the dual (attention-like) mode, Sec. 3.4.2 / Sec. 5.1: build
   the T x T semiseparable matrix M[i, j] = C_i . (a_{j+1} ... a_i) B_j delta_j
   (lower triangle) explicitly and multiply. numpy, tiny sizes only. It pins the
@@ -68,6 +70,11 @@ def _load():
                                           fp, fp, fp, fp, fp, fp, fp,
                                           ctypes.c_int, i32p, i32p, i64p, dp, dp, ctypes.c_int]
             lib.ssd_ref_max_threads.restype = ctypes.c_int
+            lib.ssd_ref_bwd.restype = ctypes.c_int
+            lib.ssd_ref_bwd.argtypes = [ctypes.c_int, i64p, i64p, ctypes.c_int, ctypes.c_int,
+                                        ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                        fp, fp, fp, fp, fp, fp, fp, fp, fp, ctypes.c_int64,
+                                        dp, dp, dp, dp, dp, dp, dp, ctypes.c_int]
             _lib = lib
     return _lib
 
@@ -145,6 +152,44 @@ def recurrence(inp: dict, nthreads: int = 0):
         y[t0:t0 + n, h, :] = ysh
     fin = np.stack(finals).reshape(len(bounds), H, P, N) if pairs else np.zeros((len(bounds), H, P, N))
     return y.reshape(x.shape), fin
+
+
+def recurrence_grad(inp: dict, dy, dfinal=None, nthreads: int = 0) -> dict:
+    """Reverse mode of the recurrence (fp64, plain C): the gradients of
+    L = <dy, y> + <dfinal, final_states> with respect to x, dt (raw, before the
+    softplus), A_log, B, C, D and the initial states. Written by differentiating
+    the per-token update of Sec. 3.4.1 eq. (8) step by step (see ssd_ref.c).
+    Returns float64 arrays shaped like the inputs: dx, ddt, dA_log, dB, dC, dD,
+    dinit (dinit has the initial-state shape (nseq, H, P, N))."""
+    lib = _load()
+    x, dt, Bm, Cm = (_f32(inp[k]) for k in ("x", "dt", "B", "C"))
+    A_log, D, init = _f32(inp["A_log"]), _f32(inp.get("D")), _f32(inp.get("initial_states"))
+    dyf = _f32(dy)
+    dfin = _f32(dfinal)
+    H, P = x.shape[2], x.shape[3]
+    G, N = Bm.shape[2], Bm.shape[3]
+    bounds = seq_bounds(inp)
+    nseq = len(bounds)
+    tokens = x.shape[0] * x.shape[1]
+    starts = np.array([b[0] for b in bounds], dtype=np.int64)
+    slens = np.array([b[1] for b in bounds], dtype=np.int64)
+    out = {"dx": np.zeros((tokens, H, P)), "ddt": np.zeros((tokens, H)), "dB": np.zeros((tokens, G, N)),
+           "dC": np.zeros((tokens, G, N)), "dA_log": np.zeros(H), "dD": np.zeros(H),
+           "dinit": np.zeros((nseq, H, P, N))}
+    rc = lib.ssd_ref_bwd(nseq, _ptr(starts, ctypes.c_int64), _ptr(slens, ctypes.c_int64), H, P, N, G,
+                         int(bool(inp.get("dt_softplus", True))), _ptr(x, ctypes.c_float),
+                         _ptr(dt, ctypes.c_float), _ptr(A_log, ctypes.c_float), _ptr(Bm, ctypes.c_float),
+                         _ptr(Cm, ctypes.c_float), _ptr(D, ctypes.c_float), _ptr(init, ctypes.c_float),
+                         _ptr(dyf, ctypes.c_float), _ptr(dfin, ctypes.c_float), tokens,
+                         *(_ptr(out[k], ctypes.c_double) for k in ("dx", "ddt", "dB", "dC", "dA_log", "dD", "dinit")),
+                         int(nthreads))
+    if rc != 0:
+        raise ValueError("ssd_ref_bwd rejected its arguments")
+    out["dx"] = out["dx"].reshape(x.shape)
+    out["ddt"] = out["ddt"].reshape(dt.shape)
+    out["dB"] = out["dB"].reshape(Bm.shape)
+    out["dC"] = out["dC"].reshape(Cm.shape)
+    return out
 
 
 def _softplus(r):

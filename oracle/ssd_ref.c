@@ -155,3 +155,194 @@ int ssd_ref_max_threads(void)
     return 1;
 #endif
 }
+
+/*
+ * Reverse mode of the same recurrence (the gradient of a loss L with respect
+ * to every input, given dL/dy and dL/dfinal_state), written by differentiating
+ * the per-token update above step by step.  With G_t = dL/dstate_t (P x N):
+ *
+ *   G_t = dy_t (outer) C_t + a_{t+1} G_{t+1},     G_T = dL/dfinal (or 0), a_T = 1
+ *   dC_t   += state_t^T dy_t                        (N; summed over the heads of a group)
+ *   dx_t    = D dy_t + delta_t G_t B_t               (P)
+ *   dB_t   += delta_t G_t^T x_t                     (N; summed over the heads of a group)
+ *   ddelta  = x_t^T G_t B_t + A a_t <G_t, state_{t-1}>
+ *   dA     += delta_t a_t <G_t, state_{t-1}>,   dA_log = A dA   (A = -exp(A_log))
+ *   dD     += <dy_t, x_t>
+ *   ddt_t   = ddelta * sigmoid(dt_t)   (ddelta when dt_softplus == 0)
+ *   dinit   = a_0 G_0
+ *
+ * state_{t-1} is needed in reverse order: states are recomputed forward from
+ * checkpoints kept every kCk tokens.
+ */
+enum { kCk = 64 };
+
+static double sigmoid(double r)
+{
+    return r >= 0.0 ? 1.0 / (1.0 + exp(-r)) : exp(r) / (1.0 + exp(r));
+}
+
+/* One (sequence, head) pair.  dB_out, dC_out: len * N doubles (this head's
+ * contribution); dx_out len * P; ddt_out len; dinit_out P * N (may be NULL). */
+static int ssd_ref_bwd_one(int64_t tok0, int64_t len, int h, int H, int P, int N, int G,
+                           int dt_softplus, const float *x, const float *dt,
+                           const float *A_log, const float *B, const float *C,
+                           const float *D, const float *init_sh, const float *dy,
+                           const float *dfin_sh, double *dx_out, double *ddt_out,
+                           double *dB_out, double *dC_out, double *dAlog_out,
+                           double *dD_out, double *dinit_out)
+{
+    const int g = h / (H / G);
+    const double A = -exp((double)A_log[h]);
+    const double Dh = D ? (double)D[h] : 0.0;
+    const int64_t PN = (int64_t)P * N;
+    const int64_t nck = (len + kCk - 1) / kCk;
+    double *ck = (double *)calloc((size_t)((nck > 0 ? nck : 1) * PN), sizeof(double));
+    double *seg = (double *)malloc(sizeof(double) * (size_t)(kCk * PN));
+    double *gst = (double *)malloc(sizeof(double) * (size_t)PN);
+    if (!ck || !seg || !gst) {
+        free(ck); free(seg); free(gst);
+        return -1;
+    }
+    /* forward: checkpoint k holds the state before token k * kCk */
+    double *st = gst;   /* scratch for the forward sweep */
+    for (int64_t i = 0; i < PN; ++i) st[i] = init_sh ? (double)init_sh[i] : 0.0;
+    for (int64_t t = 0; t < len; ++t) {
+        if (t % kCk == 0) memcpy(ck + (t / kCk) * PN, st, sizeof(double) * (size_t)PN);
+        const int64_t tok = tok0 + t;
+        const double r = (double)dt[tok * H + h];
+        const double delta = dt_softplus ? softplus(r) : r;
+        const double a = exp(delta * A);
+        const float *xt = x + (tok * H + h) * (int64_t)P;
+        const float *Bt = B + (tok * G + g) * (int64_t)N;
+        for (int p = 0; p < P; ++p)
+            for (int n = 0; n < N; ++n)
+                st[(int64_t)p * N + n] = a * st[(int64_t)p * N + n] + delta * (double)xt[p] * (double)Bt[n];
+    }
+    /* reverse sweep; gst = a_{t+1} G_{t+1} before step t */
+    for (int64_t i = 0; i < PN; ++i) gst[i] = dfin_sh ? (double)dfin_sh[i] : 0.0;
+    double dA = 0.0, dDh = 0.0;
+    for (int64_t k = nck - 1; k >= 0; --k) {
+        const int64_t t0 = k * kCk, t1 = (t0 + kCk < len) ? t0 + kCk : len;
+        /* recompute state_t for t in [t0, t1): seg[t - t0] */
+        for (int64_t t = t0; t < t1; ++t) {
+            const int64_t tok = tok0 + t;
+            const double r = (double)dt[tok * H + h];
+            const double delta = dt_softplus ? softplus(r) : r;
+            const double a = exp(delta * A);
+            const float *xt = x + (tok * H + h) * (int64_t)P;
+            const float *Bt = B + (tok * G + g) * (int64_t)N;
+            const double *prev = (t == t0) ? ck + k * PN : seg + (t - 1 - t0) * PN;
+            double *cur = seg + (t - t0) * PN;
+            for (int p = 0; p < P; ++p)
+                for (int n = 0; n < N; ++n)
+                    cur[(int64_t)p * N + n] = a * prev[(int64_t)p * N + n] + delta * (double)xt[p] * (double)Bt[n];
+        }
+        for (int64_t t = t1 - 1; t >= t0; --t) {
+            const int64_t tok = tok0 + t;
+            const double r = (double)dt[tok * H + h];
+            const double delta = dt_softplus ? softplus(r) : r;
+            const double a = exp(delta * A);
+            const float *xt = x + (tok * H + h) * (int64_t)P;
+            const float *dyt = dy + (tok * H + h) * (int64_t)P;
+            const float *Bt = B + (tok * G + g) * (int64_t)N;
+            const float *Ct = C + (tok * G + g) * (int64_t)N;
+            const double *cur = seg + (t - t0) * PN;
+            const double *prev = (t == t0) ? ck + k * PN : seg + (t - 1 - t0) * PN;
+            double ddelta = 0.0, gh = 0.0;
+            for (int p = 0; p < P; ++p) {
+                const double dyp = (double)dyt[p], xp = (double)xt[p];
+                double gb = 0.0;
+                for (int n = 0; n < N; ++n) {
+                    double *gp = gst + (int64_t)p * N + n;
+                    *gp += dyp * (double)Ct[n];                 /* G_t */
+                    gb += *gp * (double)Bt[n];
+                    gh += *gp * prev[(int64_t)p * N + n];
+                    dC_out[(t)*N + n] += dyp * cur[(int64_t)p * N + n];
+                    dB_out[(t)*N + n] += delta * xp * *gp;
+                }
+                dx_out[t * P + p] = Dh * dyp + delta * gb;
+                ddelta += xp * gb;
+                dDh += dyp * xp;
+            }
+            ddelta += A * a * gh;
+            dA += delta * a * gh;
+            ddt_out[t] = dt_softplus ? ddelta * sigmoid(r) : ddelta;
+            for (int64_t i = 0; i < PN; ++i) gst[i] *= a;   /* a_t G_t, for step t - 1 */
+        }
+    }
+    if (dinit_out) memcpy(dinit_out, gst, sizeof(double) * (size_t)PN);
+    *dAlog_out = A * dA;
+    *dD_out = dDh;
+    free(ck); free(seg); free(gst);
+    return 0;
+}
+
+/*
+ * Gradients for every (sequence, head) pair of a batch.  Inputs as for
+ * ssd_ref_pairs plus dy (tokens, H, P) and dfinal (nseq, H, P, N, may be
+ * NULL).  Outputs (double, zeroed here): dx (tokens, H, P), ddt (tokens, H),
+ * dB and dC (tokens, G, N), dA_log and dD (H), dinit (nseq, H, P, N).
+ */
+int ssd_ref_bwd(int nseq, const int64_t *seq_start, const int64_t *seq_len,
+                int H, int P, int N, int G, int dt_softplus,
+                const float *x, const float *dt, const float *A_log,
+                const float *B, const float *C, const float *D, const float *init,
+                const float *dy, const float *dfinal, int64_t tokens,
+                double *dx, double *ddt, double *dB, double *dC, double *dA_log,
+                double *dD, double *dinit, int nthreads)
+{
+    if (nseq < 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0 || H % G != 0 || tokens < 0)
+        return -1;
+    if (!x || !dt || !A_log || !B || !C || !dy || !dx || !ddt || !dB || !dC || !dA_log || !dD || !dinit)
+        return -1;
+    const int64_t PN = (int64_t)P * N;
+    memset(dx, 0, sizeof(double) * (size_t)(tokens * H * P));
+    memset(ddt, 0, sizeof(double) * (size_t)(tokens * H));
+    memset(dB, 0, sizeof(double) * (size_t)(tokens * G * N));
+    memset(dC, 0, sizeof(double) * (size_t)(tokens * G * N));
+    memset(dA_log, 0, sizeof(double) * (size_t)H);
+    memset(dD, 0, sizeof(double) * (size_t)H);
+    memset(dinit, 0, sizeof(double) * (size_t)(nseq * H * PN));
+    int bad = 0;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    const int npairs = nseq * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int i = 0; i < npairs; ++i) {
+        const int s = i / H, h = i % H, g = h / (H / G);
+        const int64_t t0 = seq_start[s], len = seq_len[s];
+        double *px = (double *)malloc(sizeof(double) * (size_t)((len > 0 ? len : 1) * P));
+        double *pdt = (double *)malloc(sizeof(double) * (size_t)(len > 0 ? len : 1));
+        double *pB = (double *)calloc((size_t)((len > 0 ? len : 1) * N), sizeof(double));
+        double *pC = (double *)calloc((size_t)((len > 0 ? len : 1) * N), sizeof(double));
+        double dal = 0.0, dd = 0.0;
+        const float *init_sh = init ? init + ((int64_t)s * H + h) * PN : NULL;
+        const float *dfin_sh = dfinal ? dfinal + ((int64_t)s * H + h) * PN : NULL;
+        if (!px || !pdt || !pB || !pC ||
+            ssd_ref_bwd_one(t0, len, h, H, P, N, G, dt_softplus, x, dt, A_log, B, C, D, init_sh, dy,
+                            dfin_sh, px, pdt, pB, pC, &dal, &dd, dinit + ((int64_t)s * H + h) * PN) != 0) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+            for (int64_t t = 0; t < len; ++t) {
+                for (int p = 0; p < P; ++p) dx[((t0 + t) * H + h) * P + p] = px[t * P + p];
+                ddt[(t0 + t) * H + h] = pdt[t];
+                for (int n = 0; n < N; ++n) {
+#pragma omp atomic
+                    dB[((t0 + t) * G + g) * N + n] += pB[t * N + n];
+#pragma omp atomic
+                    dC[((t0 + t) * G + g) * N + n] += pC[t * N + n];
+                }
+            }
+#pragma omp atomic
+            dA_log[h] += dal;
+#pragma omp atomic
+            dD[h] += dd;
+        }
+        free(px); free(pdt); free(pB); free(pC);
+    }
+    return bad ? -1 : 0;
+}
