@@ -207,6 +207,42 @@ SSD_API ssd_status ssd_decode_step(const ssd_step_params *p,
                    const void *B, const void *C, const float *D,
                    float *state, void *y, void *stream);
 
+/* Backward pass: the gradients of a loss L given dy = dL/dy and
+ * dfinal_states = dL/dfinal_states, for training ("Transformers are SSMs",
+ * Thm. 6.1 counts the training cost of the SSD algorithm; the gradient is the
+ * same block decomposition of Sec. 6 run in reverse).  With the forward's
+ * per-token update (see the top of this file) and G_t = dL/dstate_t:
+ *
+ *     G_t = dy_t (outer) C_t + a_{t+1} G_{t+1},   G_last = dL/dfinal_states
+ *     dx_t = D dy_t + delta_t G_t B_t,   dB_t = sum over the group's heads of delta_t G_t^T x_t,
+ *     dC_t = sum over the group's heads of state_t^T dy_t,
+ *     ddelta_t = x_t^T G_t B_t + A a_t <G_t, state_{t-1}>,   ddt_t = ddelta_t sigmoid(dt_t)
+ *     (ddelta_t itself when dt_softplus == 0),   dA_log = A sum_t delta_t a_t <G_t, state_{t-1}>,
+ *     dD = sum_t <dy_t, x_t>,   dinitial_states = a_first G_first
+ *
+ * Inputs are those of ssd_fwd plus dy (y's layout and io dtype) and
+ * dfinal_states ((nseq, nheads, headdim, dstate) float32, NULL = 0).
+ * Every gradient is float32, in the layout of its input: dx (batch, seqlen,
+ * nheads, headdim), ddt (batch, seqlen, nheads) with respect to the raw dt,
+ * dA_log and dD (nheads), dB and dC (batch, seqlen, ngroups, dstate),
+ * dinitial_states (nseq, nheads, headdim, dstate; NULL: not written).  D and
+ * initial_states may be NULL as in ssd_fwd; dD is written either way.  The
+ * pass recomputes the forward's chunk states on CUDA cores with 32-token
+ * chunks (chunk_len is not used; the result does not depend on it) and holds
+ * two fp32 states per chunk and head in the workspace.  Supported: float32
+ * or bf16 inputs, headdim <= 128, dstate <= 256, path AUTO or SIMT
+ * (SSD_PATH_TENSOR returns SSD_ERR_UNSUPPORTED).  Errors and asynchrony as
+ * for ssd_fwd; ssd_get_status reads the workspace's status word. */
+SSD_API size_t ssd_bwd_workspace_size(const ssd_fwd_params *p);
+
+SSD_API ssd_status ssd_bwd(const ssd_fwd_params *p,
+                   const void *x, const void *dt, const float *A_log,
+                   const void *B, const void *C, const float *D,
+                   const float *initial_states, const int32_t *cu_seqlens,
+                   const void *dy, const float *dfinal_states,
+                   float *dx, float *ddt, float *dA_log, float *dB, float *dC, float *dD,
+                   float *dinitial_states, void *workspace, size_t workspace_bytes, void *stream);
+
 /* Device-side status of the last ssd_fwd that used `workspace` on `stream`:
  * synchronises `stream`, then returns SSD_OK, SSD_ERR_TIMEOUT or
  * SSD_ERR_BAD_SEQLENS (or SSD_ERR_CUDA if the copy fails). */

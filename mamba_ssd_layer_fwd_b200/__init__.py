@@ -22,7 +22,7 @@ import threading
 from typing import Optional
 
 __all__ = [
-    "ssd_fwd", "ssd_decode_step", "SsdParams", "SsdStepParams", "SsdInstrumentation", "make_instrumentation", "workspace_size",
+    "ssd_fwd", "ssd_bwd", "ssd_decode_step", "SsdParams", "SsdStepParams", "SsdInstrumentation", "make_instrumentation", "workspace_size",
     "launch_count", "resolved_path", "library", "library_path", "STATUS", "PATHS", "SsdError",
 ]
 
@@ -36,7 +36,7 @@ STATUS = {0: "SSD_OK", -1: "SSD_ERR_INVALID_ARG", -2: "SSD_ERR_UNSUPPORTED", -3:
 PATHS = {"auto": 0, "simt": 1, "tensor": 2}
 DTYPES = {"f32": 0, "bf16": 1}
 
-EXPORTED = ("ssd_fwd", "ssd_fwd_instrumented", "ssd_decode_step", "ssd_fwd_workspace_size", "ssd_get_status", "ssd_fwd_launch_count",
+EXPORTED = ("ssd_fwd", "ssd_fwd_instrumented", "ssd_bwd", "ssd_bwd_workspace_size", "ssd_decode_step", "ssd_fwd_workspace_size", "ssd_get_status", "ssd_fwd_launch_count",
             "ssd_fwd_resolved_path", "ssd_status_string", "ssd_abi_version")
 
 
@@ -91,6 +91,10 @@ def library():
             lib.ssd_fwd_instrumented.restype = i32
             lib.ssd_fwd_instrumented.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
                                                  ctypes.POINTER(SsdInstrumentation)]
+            lib.ssd_bwd.restype = i32
+            lib.ssd_bwd.argtypes = [pp] + [vp] * 17 + [vp, sz, vp]
+            lib.ssd_bwd_workspace_size.restype = sz
+            lib.ssd_bwd_workspace_size.argtypes = [pp]
             lib.ssd_decode_step.restype = i32
             lib.ssd_decode_step.argtypes = [ctypes.POINTER(SsdStepParams), vp, vp, vp, vp, vp, vp, vp, vp, vp]
             lib.ssd_fwd_workspace_size.restype = sz
@@ -229,6 +233,55 @@ def ssd_fwd(x, dt, A_log, B, C, D=None, chunk_len: int = 256, initial_states=Non
         if rc != 0:
             raise SsdError(rc, "ssd_fwd (device status)")
     return (y, final_states) if want_final else y
+
+
+def ssd_bwd(x, dt, A_log, B, C, D, dy, initial_states=None, cu_seqlens=None, dfinal_states=None,
+            dt_softplus: bool = True, want_dinitial: bool = True, workspace=None, stream=None,
+            check_status: bool = False) -> dict:
+    """Gradients of L given dy = dL/dy (and dL/dfinal_states) through the C ABI.
+    Returns float32 tensors: dx, ddt (with respect to the raw dt), dA_log, dB,
+    dC, dD and dinitial_states (when `want_dinitial`), each shaped like its input."""
+    import torch
+    lib = library()
+    dev = x.device
+    if dev.type != "cuda":
+        raise ValueError("ssd_bwd runs on CUDA tensors only")
+    for name, t in (("x", x), ("dt", dt), ("B", B), ("C", C), ("dy", dy)):
+        if t.dtype != x.dtype or not t.is_contiguous() or t.device != dev:
+            raise ValueError(f"{name} must be a contiguous {x.dtype} tensor on {dev}")
+    for name, t in (("A_log", A_log), ("D", D), ("initial_states", initial_states),
+                    ("dfinal_states", dfinal_states)):
+        if t is not None and (t.dtype != torch.float32 or not t.is_contiguous() or t.device != dev):
+            raise ValueError(f"{name} must be a contiguous float32 tensor on {dev}")
+    if dy.shape != x.shape:
+        raise ValueError("dy must have x's shape")
+    p = params_for(x, B, 256, cu_seqlens, dt_softplus, "auto")
+    b, T, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    nseq = p.num_seqs if p.num_seqs > 0 else b
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = {"dx": torch.empty(x.shape, **f32), "ddt": torch.empty(dt.shape, **f32),
+           "dA_log": torch.empty(H, **f32), "dB": torch.empty(B.shape, **f32), "dC": torch.empty(C.shape, **f32),
+           "dD": torch.empty(H, **f32),
+           "dinitial_states": torch.empty((nseq, H, P, N), **f32) if want_dinitial else None}
+    need = int(lib.ssd_bwd_workspace_size(ctypes.byref(p)))
+    if need == 0:
+        raise SsdError(-2, "ssd_bwd_workspace_size")
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    st = _stream_handle(stream)
+    rc = lib.ssd_bwd(ctypes.byref(p), _ptr(x), _ptr(dt), _ptr(A_log), _ptr(B), _ptr(C), _ptr(D),
+                     _ptr(initial_states), _ptr(cu_seqlens), _ptr(dy), _ptr(dfinal_states),
+                     _ptr(out["dx"]), _ptr(out["ddt"]), _ptr(out["dA_log"]), _ptr(out["dB"]), _ptr(out["dC"]),
+                     _ptr(out["dD"]), _ptr(out["dinitial_states"]), _ptr(workspace),
+                     workspace.numel() * workspace.element_size(), st)
+    if rc != 0:
+        raise SsdError(rc, "ssd_bwd")
+    if check_status:
+        rc = lib.ssd_get_status(_ptr(workspace), st)
+        if rc != 0:
+            raise SsdError(rc, "ssd_bwd (device status)")
+    return out
 
 
 def ssd_decode_step(x, dt, A_log, B, C, D, state, y=None, dt_softplus: bool = True, stream=None):

@@ -223,6 +223,95 @@ ssd_status ssd_fwd_instrumented(const ssd_fwd_params *p, const void *x, const vo
     }
 }
 
+namespace {
+
+struct BwdLayout {
+    size_t status, count, chunks, seqs, cs, dv, states, gbuf, total;
+};
+
+BwdLayout bwd_layout(const ssd_fwd_params &p)
+{
+    BwdLayout L{};
+    size_t off = 0;
+    const size_t mc = bwd_chunk_count(p), ns = (size_t)nseq_of(p), Q = (size_t)bwd_chunk_len();
+    const size_t pn = (size_t)p.headdim * p.dstate;
+    L.status = off; off += kAlign;
+    L.count = off; off += kAlign;
+    L.chunks = off; off = align_up(off + mc * sizeof(ChunkDesc));
+    L.seqs = off; off = align_up(off + ns * sizeof(SeqDesc));
+    L.cs = off; off = align_up(off + mc * p.nheads * Q * sizeof(float));
+    L.dv = off; off = align_up(off + mc * p.nheads * Q * sizeof(float));
+    L.states = off; off = align_up(off + mc * p.nheads * pn * sizeof(float));
+    L.gbuf = off; off = align_up(off + mc * p.nheads * pn * sizeof(float));
+    L.total = off;
+    return L;
+}
+
+}  // namespace
+
+size_t ssd_bwd_workspace_size(const ssd_fwd_params *p)
+{
+    if (validate(p) != SSD_OK || !bwd_supported(*p)) return 0;
+    return bwd_layout(*p).total;
+}
+
+ssd_status ssd_bwd(const ssd_fwd_params *p, const void *x, const void *dt, const float *A_log, const void *B,
+                   const void *C, const float *D, const float *initial_states, const int32_t *cu_seqlens,
+                   const void *dy, const float *dfinal_states, float *dx, float *ddt, float *dA_log, float *dB,
+                   float *dC, float *dD, float *dinitial_states, void *workspace, size_t workspace_bytes,
+                   void *stream)
+{
+    try {
+        const ssd_status v = validate(p);
+        if (v != SSD_OK) return v;
+        if (!bwd_supported(*p)) return SSD_ERR_UNSUPPORTED;
+        const bool has_tokens = (long long)p->batch * p->seqlen > 0;
+        if (!A_log || !workspace || !dA_log || !dD) return SSD_ERR_INVALID_ARG;
+        if (has_tokens && (!x || !dt || !B || !C || !dy || !dx || !ddt || !dB || !dC)) return SSD_ERR_INVALID_ARG;
+        if ((p->num_seqs > 0) != (cu_seqlens != nullptr)) return SSD_ERR_INVALID_ARG;
+        const void *ptrs[] = {x, dt, A_log, B, C, D, initial_states, cu_seqlens, dy, dfinal_states, dx, ddt,
+                              dA_log, dB, dC, dD, dinitial_states};
+        for (const void *q : ptrs)
+            if (q && !aligned16(q)) return SSD_ERR_INVALID_ARG;
+        if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0) return SSD_ERR_INVALID_ARG;
+        const BwdLayout L = bwd_layout(*p);
+        if (workspace_bytes < L.total) return SSD_ERR_INVALID_ARG;
+
+        cudaStream_t st = static_cast<cudaStream_t>(stream);
+        char *ws = static_cast<char *>(workspace);
+        Plan plan;
+        plan.status = reinterpret_cast<int *>(ws + L.status);
+        plan.count = reinterpret_cast<int *>(ws + L.count);
+        plan.chunks = reinterpret_cast<ChunkDesc *>(ws + L.chunks);
+        plan.seqs = reinterpret_cast<SeqDesc *>(ws + L.seqs);
+        plan.nseq = nseq_of(*p);
+        plan.max_chunks = (int)bwd_chunk_count(*p);
+        Dims d;
+        d.H = p->nheads;
+        d.P = p->headdim;
+        d.N = p->dstate;
+        d.G = p->ngroups;
+        d.Q = bwd_chunk_len();
+        d.heads_per_group = p->nheads / p->ngroups;
+        d.tokens = p->batch * p->seqlen;
+        d.dt_softplus = p->dt_softplus;
+        if (launch_build_plan(plan, cu_seqlens, p->batch, p->seqlen, d.Q, st) != cudaSuccess) return SSD_ERR_CUDA;
+        SimtArgs fa;
+        fa.x = x; fa.dt = dt; fa.B = B; fa.C = C;
+        fa.A_log = A_log; fa.D = D; fa.init = initial_states;
+        fa.y = nullptr; fa.final_states = nullptr;
+        fa.cs = reinterpret_cast<float *>(ws + L.cs);
+        fa.dv = reinterpret_cast<float *>(ws + L.dv);
+        fa.states = reinterpret_cast<float *>(ws + L.states);
+        fa.bf16 = p->io_dtype == SSD_DTYPE_BF16;
+        const cudaError_t e = launch_bwd(plan, d, fa, dy, dfinal_states, reinterpret_cast<float *>(ws + L.gbuf), dx,
+                                         ddt, dA_log, dB, dC, dD, dinitial_states, fa.bf16, st);
+        return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+    } catch (...) {
+        return SSD_ERR_CUDA;
+    }
+}
+
 ssd_status ssd_get_status(const void *workspace, void *stream)
 {
     if (!workspace) return SSD_ERR_INVALID_ARG;

@@ -1,0 +1,415 @@
+// Backward pass of the SSD layer on CUDA cores (fp32 arithmetic): the chunked
+// block decomposition of "Transformers are SSMs", Sec. 6, run in reverse.
+//
+// With 32-token chunks c, per head: cs_l the inclusive cumsum of delta * A
+// inside the chunk, H_c the state entering chunk c (recomputed with the
+// forward's cumsum / chunk-state / state-passing kernels), and G_c = dL/dH_c:
+//
+//   U_c      = sum_l exp(cs_l) dy_l (outer) C_l                      (dstate kernel)
+//   G_c      = U_c + exp(cs_last) G_{c+1},  G_nc = dL/dfinal,  dL/dinit = G_0
+//                                                                    (reverse state passing)
+// and inside chunk c (L[l,s] = exp(cs_l - cs_s) for s <= l, W = L o C B^T,
+// e2_s = exp(cs_last - cs_s), Gn = G_{c+1}):
+//
+//   dx_s  = D dy_s + delta_s (sum_l W[l,s] dy_l + e2_s Gn B_s)
+//   dB_s  = delta_s (sum_l L[l,s] (dy_l . x_s) C_l + e2_s Gn^T x_s)   (summed over the group's heads)
+//   dC_l  = sum_s L[l,s] delta_s (dy_l . x_s) B_s + exp(cs_l) H_c^T dy_l
+//   dcs_l = sum_{s<l} E[l,s] - sum_{l'>l} E[l',l] + exp(cs_l) dy_l . (H_c C_l) - F_l
+//           + [l last] (sum_s F_s + exp(cs_last) <Gn, H_c>),
+//           E[l,s] = W[l,s] delta_s (dy_l . x_s),  F_s = e2_s delta_s x_s . (Gn B_s)
+//   d(dA)_k = sum_{l >= k} dcs_l          (dA = delta * A enters cs_l for every l >= k)
+//   ddelta_k = A d(dA)_k + sum_l W[l,k] (dy_l . x_k) + e2_k x_k . (Gn B_k)
+//   ddt = ddelta * sigmoid(dt) (softplus), dA_log = A sum_k delta_k d(dA)_k, dD = sum <dy, x>
+//
+// Every exponent above is a difference cs_l - cs_s with s <= l, <= 0 in exact
+// arithmetic; the fp32 prefix sums can round it above 0 when |A| is huge, so
+// it is clamped at 0.
+//
+// One CTA per (chunk, B/C group) loops over the group's heads, keeping the
+// group's dB and dC tiles in shared memory, so they are written once, without
+// atomics; dA_log and dD are summed with one atomic per (chunk, head).
+#include "ssd_common.cuh"
+
+namespace ssd {
+namespace {
+
+constexpr int kBQ = 32;         // chunk length of the backward
+constexpr int kBThreads = 256;
+constexpr int kNT = 32;         // dstate columns per tile of H_c and G_{c+1}
+
+__device__ __forceinline__ float sigmoid_f32(float r)
+{
+    // 1 / (1 + e^-r), evaluated without overflow
+    const float e = __expf(-fabsf(r));
+    return r >= 0.0f ? 1.0f / (1.0f + e) : e / (1.0f + e);
+}
+
+// U_c[p][n] = sum_l exp(cs_l) dy_l[p] C_l[n], written into `ubuf` (the layout of the chunk states)
+template <typename T>
+__global__ void __launch_bounds__(kBThreads)
+bwd_dstate_kernel(Plan plan, Dims d, const T *__restrict__ dy, const T *__restrict__ Cm,
+                  const float *__restrict__ cs, float *__restrict__ ubuf)
+{
+    extern __shared__ float smem[];
+    const int c = blockIdx.x;
+    if (c >= *plan.count) return;
+    const ChunkDesc ch = plan.chunks[c];
+    const int h = blockIdx.y, g = h / d.heads_per_group;
+    const int P = d.P, N = d.N;
+    float *Ys = smem;                 // kBQ x P (weighted dy)
+    float *Cs = Ys + kBQ * P;         // kBQ x N
+    const float *csc = cs + ((size_t)c * d.H + h) * kBQ;
+    for (int i = threadIdx.x; i < kBQ * P; i += kBThreads) {
+        const int l = i / P, p = i % P;
+        Ys[i] = l < ch.len ? __expf(csc[l]) * to_f32(dy[((size_t)(ch.tok0 + l) * d.H + h) * P + p]) : 0.0f;
+    }
+    for (int i = threadIdx.x; i < kBQ * N; i += kBThreads) {
+        const int l = i / N, n = i % N;
+        Cs[i] = l < ch.len ? to_f32(Cm[((size_t)(ch.tok0 + l) * d.G + g) * N + n]) : 0.0f;
+    }
+    __syncthreads();
+    const int PN = P * N;
+    float *out = ubuf + ((size_t)c * d.H + h) * PN;
+    for (int e = threadIdx.x; e < PN; e += kBThreads) {
+        const int p = e / N, n = e % N;
+        float a = 0.0f;
+#pragma unroll 8
+        for (int l = 0; l < kBQ; ++l) a = fmaf(Ys[l * P + p], Cs[l * N + n], a);
+        out[e] = a;
+    }
+}
+
+// G_c = U_c + exp(cs_last(c)) G_{c+1} from the last chunk of each sequence to
+// the first; the buffer slot of chunk c receives G_{c+1} (dL/d of the state
+// leaving the chunk), and dL/dinit = G_0.
+__global__ void __launch_bounds__(kBThreads)
+bwd_state_passing_kernel(Plan plan, Dims d, const float *__restrict__ cs, float *__restrict__ gbuf,
+                         const float *__restrict__ dfinal, float *__restrict__ dinit)
+{
+    const int s = blockIdx.x, h = blockIdx.y;
+    const int PN = d.P * d.N;
+    const int e = blockIdx.z * kBThreads + threadIdx.x;
+    if (e >= PN) return;
+    const SeqDesc sq = plan.seqs[s];
+    float gv = dfinal ? dfinal[((size_t)s * d.H + h) * PN + e] : 0.0f;
+    for (int j = sq.nchunks - 1; j >= 0; --j) {
+        const int c = sq.chunk0 + j;
+        const size_t idx = ((size_t)c * d.H + h) * PN + e;
+        const float u = gbuf[idx];
+        gbuf[idx] = gv;
+        const float decay = __expf(cs[((size_t)c * d.H + h) * kBQ + kBQ - 1]);
+        gv = fmaf(decay, gv, u);
+    }
+    if (dinit) dinit[((size_t)s * d.H + h) * PN + e] = gv;
+}
+
+struct BwdArgs {
+    const void *x, *dt, *B, *C, *dy;
+    const float *A_log, *D;
+    const float *cs, *dv, *states, *gbuf;
+    float *dx, *ddt, *dA_log, *dB, *dC, *dD;
+};
+
+size_t chunk_smem_floats(int P, int N)
+{
+    const int PS = P + 1, NS = N + 1, QS = kBQ + 1;
+    return (size_t)2 * kBQ * NS        // B, C
+           + 2 * kBQ * NS              // dB, dC accumulators
+           + 2 * kBQ * PS              // x, dy
+           + 3 * kBQ * QS              // C B^T, L, dy . x
+           + 2 * P * (kNT + 1)         // H_c, G_{c+1} tiles
+           + 8 * kBQ + 32;             // per-token vectors, reductions
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kBThreads)
+bwd_chunk_kernel(Plan plan, Dims d, BwdArgs a)
+{
+    extern __shared__ float smem[];
+    const int c = blockIdx.x;
+    if (c >= *plan.count) return;
+    const ChunkDesc ch = plan.chunks[c];
+    const int g = blockIdx.y;
+    const int P = d.P, N = d.N, H = d.H, G = d.G;
+    const int PS = P + 1, NS = N + 1, QS = kBQ + 1;
+    const int len = ch.len;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    float *Bs = smem;                      // kBQ x NS
+    float *Cs = Bs + kBQ * NS;
+    float *dBs = Cs + kBQ * NS;            // group accumulators
+    float *dCs = dBs + kBQ * NS;
+    float *Xs = dCs + kBQ * NS;            // kBQ x PS (current head)
+    float *DYs = Xs + kBQ * PS;
+    float *CB = DYs + kBQ * PS;            // kBQ x QS: C_l . B_s
+    float *Lm = CB + kBQ * QS;             // exp(cs_l - cs_s), s <= l < len
+    float *DX = Lm + kBQ * QS;             // dy_l . x_s
+    float *Ht = DX + kBQ * QS;             // P x (kNT + 1)
+    float *Gt = Ht + P * (kNT + 1);
+    float *css = Gt + P * (kNT + 1);       // kBQ
+    float *dls = css + kBQ;                // delta (0 past the chunk's end)
+    float *fxs = dls + kBQ;                // x_s . (Gn B_s)
+    float *dhc = fxs + kBQ;                // dy_l . (H C_l)
+    float *rowv = dhc + kBQ;
+    float *colv = rowv + kBQ;
+    float *red = colv + kBQ;               // [0] <Gn, H>, [1] dD partial
+
+    const T *x = static_cast<const T *>(a.x), *dy = static_cast<const T *>(a.dy);
+    const T *Bm = static_cast<const T *>(a.B), *Cm = static_cast<const T *>(a.C);
+    const T *dtp = static_cast<const T *>(a.dt);
+
+    for (int i = tid; i < kBQ * N; i += kBThreads) {
+        const int r = i / N, n = i % N;
+        const bool v = r < len;
+        const size_t o = ((size_t)(ch.tok0 + r) * G + g) * N + n;
+        Bs[r * NS + n] = v ? to_f32(Bm[o]) : 0.0f;
+        Cs[r * NS + n] = v ? to_f32(Cm[o]) : 0.0f;
+        dBs[r * NS + n] = 0.0f;
+        dCs[r * NS + n] = 0.0f;
+    }
+    __syncthreads();
+    // C_l . B_s for the whole group
+    for (int i = tid; i < kBQ * kBQ; i += kBThreads) {
+        const int l = i / kBQ, s = i % kBQ;
+        float v = 0.0f;
+        for (int n = 0; n < N; ++n) v = fmaf(Cs[l * NS + n], Bs[s * NS + n], v);
+        CB[l * QS + s] = v;
+    }
+
+    constexpr int kMaxOut = kBQ * 128 / kBThreads;   // (s, p) outputs per thread, P <= 128
+    for (int h = g * d.heads_per_group; h < (g + 1) * d.heads_per_group; ++h) {
+        const float A = -__expf(a.A_log[h]);
+        const float Dh = a.D ? a.D[h] : 0.0f;
+        const float *csc = a.cs + ((size_t)c * H + h) * kBQ;
+        const float *dvc = a.dv + ((size_t)c * H + h) * kBQ;
+        __syncthreads();   // previous head done with Xs, DYs, Lm, DX, per-token vectors
+        for (int i = tid; i < kBQ * P; i += kBThreads) {
+            const int r = i / P, p = i % P;
+            const bool v = r < len;
+            const size_t o = ((size_t)(ch.tok0 + r) * H + h) * P + p;
+            Xs[r * PS + p] = v ? to_f32(x[o]) : 0.0f;
+            DYs[r * PS + p] = v ? to_f32(dy[o]) : 0.0f;
+        }
+        if (tid < kBQ) {
+            css[tid] = csc[tid];
+            dls[tid] = tid < len ? dvc[tid] : 0.0f;
+            fxs[tid] = 0.0f;
+            dhc[tid] = 0.0f;
+        }
+        if (tid < 2) red[tid] = 0.0f;
+        __syncthreads();
+        for (int i = tid; i < kBQ * kBQ; i += kBThreads) {
+            const int l = i / kBQ, s = i % kBQ;
+            float v = 0.0f;
+            for (int p = 0; p < P; ++p) v = fmaf(DYs[l * PS + p], Xs[s * PS + p], v);
+            DX[l * QS + s] = v;
+            Lm[l * QS + s] = (s <= l && l < len) ? __expf(fminf(css[l] - css[s], 0.0f)) : 0.0f;
+        }
+        __syncthreads();
+        // per token: row and column sums of E and of W o (dy . x); dD.  The sums for d(cs)
+        // leave out the diagonal, whose terms cancel exactly (d exp(cs_l - cs_l) = 0): left in,
+        // their rounding would be multiplied by A, which can be large
+        if (tid < kBQ) {
+            const int t = tid;
+            float row = 0.0f, col = 0.0f;
+            for (int s = 0; s < t; ++s) row = fmaf(Lm[t * QS + s] * CB[t * QS + s] * DX[t * QS + s], dls[s], row);
+            for (int l = t + 1; l < kBQ; ++l) col = fmaf(Lm[l * QS + t] * CB[l * QS + t], DX[l * QS + t], col);
+            rowv[t] = row;
+            colv[t] = col;
+            float dd = t < len ? DX[t * QS + t] : 0.0f;
+            for (int o = 16; o > 0; o >>= 1) dd += __shfl_xor_sync(0xffffffffu, dd, o);
+            if (t == 0) red[1] = dd;
+        }
+        // intra terms of dx (into registers), dB, dC
+        float dxr[kMaxOut];
+#pragma unroll
+        for (int k = 0; k < kMaxOut; ++k) {
+            const int i = tid + k * kBThreads;
+            float v = 0.0f;
+            if (i < kBQ * P) {
+                const int s = i / P, p = i % P;
+                for (int l = s; l < kBQ; ++l) v = fmaf(Lm[l * QS + s] * CB[l * QS + s], DYs[l * PS + p], v);
+            }
+            dxr[k] = v;
+        }
+        for (int i = tid; i < kBQ * N; i += kBThreads) {
+            const int s = i / N, n = i % N;
+            float vb = 0.0f, vc = 0.0f;
+            for (int l = s; l < kBQ; ++l) vb = fmaf(Lm[l * QS + s] * DX[l * QS + s], Cs[l * NS + n], vb);
+            for (int t = 0; t <= s; ++t) vc = fmaf(Lm[s * QS + t] * DX[s * QS + t] * dls[t], Bs[t * NS + n], vc);
+            dBs[s * NS + n] += dls[s] * vb;
+            dCs[s * NS + n] += vc;
+        }
+        // inter terms, over tiles of kNT dstate columns of H_c and G_{c+1}
+        const float *Hc = a.states + ((size_t)c * H + h) * (size_t)P * N;
+        const float *Gn = a.gbuf + ((size_t)c * H + h) * (size_t)P * N;
+        float gbr[kMaxOut];
+#pragma unroll
+        for (int k = 0; k < kMaxOut; ++k) gbr[k] = 0.0f;
+        float ghp = 0.0f;
+        for (int n0 = 0; n0 < N; n0 += kNT) {
+            const int nt = min(kNT, N - n0);
+            __syncthreads();
+            for (int i = tid; i < P * kNT; i += kBThreads) {
+                const int p = i / kNT, nn = i % kNT;
+                const bool v = nn < nt;
+                const float hv = v ? Hc[(size_t)p * N + n0 + nn] : 0.0f;
+                const float gv = v ? Gn[(size_t)p * N + n0 + nn] : 0.0f;
+                Ht[p * (kNT + 1) + nn] = hv;
+                Gt[p * (kNT + 1) + nn] = gv;
+                ghp = fmaf(hv, gv, ghp);
+            }
+            __syncthreads();
+            // (Gn B_s)[p] over this tile
+#pragma unroll
+            for (int k = 0; k < kMaxOut; ++k) {
+                const int i = tid + k * kBThreads;
+                if (i < kBQ * P) {
+                    const int s = i / P, p = i % P;
+                    float v = gbr[k];
+                    for (int nn = 0; nn < nt; ++nn) v = fmaf(Bs[s * NS + n0 + nn], Gt[p * (kNT + 1) + nn], v);
+                    gbr[k] = v;
+                }
+            }
+            // x_s . Gn[:, n] and dy_l . H[:, n] for the tile's columns
+            for (int i = tid; i < kBQ * kNT; i += kBThreads) {
+                const int s = i / kNT, nn = i % kNT;
+                if (nn >= nt) continue;
+                float xg = 0.0f, dh = 0.0f;
+                for (int p = 0; p < P; ++p) {
+                    xg = fmaf(Xs[s * PS + p], Gt[p * (kNT + 1) + nn], xg);
+                    dh = fmaf(DYs[s * PS + p], Ht[p * (kNT + 1) + nn], dh);
+                }
+                const int n = n0 + nn;
+                const float e2 = __expf(fminf(css[kBQ - 1] - css[s], 0.0f));
+                dBs[s * NS + n] += dls[s] * e2 * xg;
+                dCs[s * NS + n] += (s < len ? __expf(css[s]) : 0.0f) * dh;
+                atomicAdd(&fxs[s], xg * Bs[s * NS + n]);
+                atomicAdd(&dhc[s], dh * Cs[s * NS + n]);
+            }
+        }
+        for (int o = 16; o > 0; o >>= 1) ghp += __shfl_xor_sync(0xffffffffu, ghp, o);
+        if (lane == 0) atomicAdd(&red[0], ghp);
+        __syncthreads();
+        // dx = D dy + delta (intra + e2 Gn B)
+#pragma unroll
+        for (int k = 0; k < kMaxOut; ++k) {
+            const int i = tid + k * kBThreads;
+            if (i < kBQ * P) {
+                const int s = i / P, p = i % P;
+                if (s < len) {
+                    const float e2 = __expf(fminf(css[kBQ - 1] - css[s], 0.0f));
+                    a.dx[((size_t)(ch.tok0 + s) * H + h) * P + p] =
+                        fmaf(Dh, DYs[s * PS + p], dls[s] * (dxr[k] + e2 * gbr[k]));
+                }
+            }
+        }
+        // d(cs) -> d(dA) (reverse cumsum) -> ddelta, ddt, dA_log, dD
+        if (warp == 0) {
+            const int t = lane;            // kBQ == 32
+            const float e2 = __expf(fminf(css[kBQ - 1] - css[t], 0.0f));
+            const float F = e2 * dls[t] * fxs[t];
+            float Fsum = F;
+            for (int o = 16; o > 0; o >>= 1) Fsum += __shfl_xor_sync(0xffffffffu, Fsum, o);
+            float dcs = rowv[t] - dls[t] * colv[t] + (t < len ? __expf(css[t]) : 0.0f) * dhc[t] - F;
+            const float colx = colv[t] + Lm[t * QS + t] * CB[t * QS + t] * DX[t * QS + t];   // with the diagonal
+            if (t == kBQ - 1) dcs += Fsum + __expf(css[kBQ - 1]) * red[0];
+            // reverse inclusive scan: ddA_k = sum_{l >= k} dcs_l
+            float v = dcs;
+            for (int o = 1; o < 32; o <<= 1) {
+                const float u = __shfl_down_sync(0xffffffffu, v, o);
+                if (t + o < 32) v += u;
+            }
+            const float ddelta = A * v + colx + e2 * fxs[t];
+            float da = dls[t] * v;
+            for (int o = 16; o > 0; o >>= 1) da += __shfl_xor_sync(0xffffffffu, da, o);
+            if (t < len) {
+                const size_t o = (size_t)(ch.tok0 + t) * H + h;
+                const float r = to_f32(dtp[o]);
+                a.ddt[o] = d.dt_softplus ? ddelta * sigmoid_f32(r) : ddelta;
+            }
+            if (t == 0) {
+                atomicAdd(&a.dA_log[h], A * da);
+                atomicAdd(&a.dD[h], red[1]);
+            }
+        }
+    }
+    __syncthreads();
+    for (int i = tid; i < len * N; i += kBThreads) {
+        const int r = i / N, n = i % N;
+        const size_t o = ((size_t)(ch.tok0 + r) * G + g) * N + n;
+        a.dB[o] = dBs[r * NS + n];
+        a.dC[o] = dCs[r * NS + n];
+    }
+}
+
+}  // namespace
+
+bool bwd_supported(const ssd_fwd_params &p)
+{
+    const size_t smem = chunk_smem_floats(p.headdim, p.dstate) * sizeof(float);
+    return p.path != SSD_PATH_TENSOR && p.headdim <= 128 && smem <= 227 * 1024;
+}
+
+size_t bwd_chunk_count(const ssd_fwd_params &p)
+{
+    const long long Q = kBQ;
+    return p.num_seqs > 0 ? (size_t)((p.seqlen + Q - 1) / Q + p.num_seqs)
+                          : (size_t)p.batch * (size_t)((p.seqlen + Q - 1) / Q);
+}
+
+int bwd_chunk_len() { return kBQ; }
+
+cudaError_t launch_bwd(const Plan &plan, const Dims &d, const SimtArgs &fa, const void *dy, const float *dfinal,
+                       float *gbuf, float *dx, float *ddt, float *dA_log, float *dB, float *dC, float *dD,
+                       float *dinit, bool bf16, cudaStream_t st)
+{
+    cudaError_t e;
+    const long long tokens = d.tokens;
+    if ((e = cudaMemsetAsync(dA_log, 0, sizeof(float) * d.H, st)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(dD, 0, sizeof(float) * d.H, st)) != cudaSuccess) return e;
+    if (tokens > 0 && (e = cudaMemsetAsync(dB, 0, sizeof(float) * tokens * d.G * d.N, st)) != cudaSuccess) return e;
+    if (tokens > 0 && (e = cudaMemsetAsync(dC, 0, sizeof(float) * tokens * d.G * d.N, st)) != cudaSuccess) return e;
+    if ((e = launch_simt_states(plan, d, fa, st)) != cudaSuccess) return e;
+    const int PN = d.P * d.N;
+    if (plan.max_chunks > 0) {
+        const dim3 gc(plan.max_chunks, d.H);
+        const size_t sd = sizeof(float) * kBQ * (d.P + d.N);
+        if (bf16) {
+            e = cudaFuncSetAttribute(bwd_dstate_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sd);
+            if (e != cudaSuccess) return e;
+            bwd_dstate_kernel<__nv_bfloat16><<<gc, kBThreads, sd, st>>>(
+                plan, d, static_cast<const __nv_bfloat16 *>(dy), static_cast<const __nv_bfloat16 *>(fa.C), fa.cs, gbuf);
+        } else {
+            e = cudaFuncSetAttribute(bwd_dstate_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sd);
+            if (e != cudaSuccess) return e;
+            bwd_dstate_kernel<float><<<gc, kBThreads, sd, st>>>(plan, d, static_cast<const float *>(dy),
+                                                                static_cast<const float *>(fa.C), fa.cs, gbuf);
+        }
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (plan.nseq > 0) {
+        const dim3 gp(plan.nseq, d.H, (PN + kBThreads - 1) / kBThreads);
+        bwd_state_passing_kernel<<<gp, kBThreads, 0, st>>>(plan, d, fa.cs, gbuf, dfinal, dinit);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (plan.max_chunks == 0) return cudaSuccess;
+    BwdArgs a;
+    a.x = fa.x; a.dt = fa.dt; a.B = fa.B; a.C = fa.C; a.dy = dy;
+    a.A_log = fa.A_log; a.D = fa.D;
+    a.cs = fa.cs; a.dv = fa.dv; a.states = fa.states; a.gbuf = gbuf;
+    a.dx = dx; a.ddt = ddt; a.dA_log = dA_log; a.dB = dB; a.dC = dC; a.dD = dD;
+    const size_t sm = chunk_smem_floats(d.P, d.N) * sizeof(float);
+    const dim3 gk(plan.max_chunks, d.G);
+    if (bf16) {
+        e = cudaFuncSetAttribute(bwd_chunk_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        if (e != cudaSuccess) return e;
+        bwd_chunk_kernel<__nv_bfloat16><<<gk, kBThreads, sm, st>>>(plan, d, a);
+    } else {
+        e = cudaFuncSetAttribute(bwd_chunk_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        if (e != cudaSuccess) return e;
+        bwd_chunk_kernel<float><<<gk, kBThreads, sm, st>>>(plan, d, a);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace ssd

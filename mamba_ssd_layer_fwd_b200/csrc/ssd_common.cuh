@@ -98,5 +98,16 @@ struct SimtArgs {
 };
 cudaError_t launch_simt(const Plan &plan, const Dims &d, const SimtArgs &a, cudaStream_t stream,
                         const Instr &ins);
+// Backward pass (ssd_bwd.cu): 32-token chunks, fp32 gradients.
+bool bwd_supported(const ssd_fwd_params &p);
+size_t bwd_chunk_count(const ssd_fwd_params &p);
+int bwd_chunk_len();
+cudaError_t launch_bwd(const Plan &plan, const Dims &d, const SimtArgs &fa, const void *dy, const float *dfinal,
+                       float *gbuf, float *dx, float *ddt, float *dA_log, float *dB, float *dC, float *dD,
+                       float *dinit, bool bf16, cudaStream_t st);
+
+// The first three SIMT kernels only (chunk cumsum, chunk states, state
+// passing): cs, dv and, in `states`, the state entering every chunk.
+cudaError_t launch_simt_states(const Plan &plan, const Dims &d, const SimtArgs &a, cudaStream_t stream);
 
 }  // namespace ssd

@@ -80,7 +80,7 @@ chunk_state_kernel(Plan plan, Dims d, const T *__restrict__ x, const T *__restri
     const float *dvc = dv + ((size_t)c * d.H + h) * Q;
     const float cs_last = csc[Q - 1];
     for (int l = threadIdx.x; l < Q; l += kThreads)
-        w[l] = l < ch.len ? __expf(cs_last - csc[l]) * dvc[l] : 0.0f;
+        w[l] = l < ch.len ? __expf(fminf(cs_last - csc[l], 0.0f)) * dvc[l] : 0.0f;   // <= 0 up to rounding
     __syncthreads();
 
     const int PN = P * N;
@@ -241,7 +241,7 @@ chunk_scan_kernel(Plan plan, Dims d, const T *__restrict__ x, const T *__restric
             if (s <= l && s < ch.len) {
                 float dot = 0.0f;
                 for (int n = 0; n < N; ++n) dot = fmaf(Cs[r * NS + n], Bs[j * NS + n], dot);
-                v = dot * __expf(csl[r] - css[j]) * dvs[j];
+                v = dot * __expf(fminf(csl[r] - css[j], 0.0f)) * dvs[j];   // s <= l: <= 0 up to rounding
             }
             Gm[r * (kTile + 1) + j] = v;
         }
@@ -315,6 +315,37 @@ cudaError_t launch_typed(const Plan &plan, const Dims &d, const SimtArgs &a, cud
 }
 
 }  // namespace
+
+cudaError_t launch_simt_states(const Plan &plan, const Dims &d, const SimtArgs &a, cudaStream_t st)
+{
+    if (plan.max_chunks == 0) return cudaSuccess;
+    const dim3 gc(plan.max_chunks, d.H);
+    const size_t ss = state_smem(d);
+    cudaError_t e;
+    if (a.bf16) {
+        chunk_cumsum_kernel<__nv_bfloat16><<<gc, d.Q, 0, st>>>(plan, d, static_cast<const __nv_bfloat16 *>(a.dt),
+                                                                a.A_log, a.cs, a.dv);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(chunk_state_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)ss);
+        if (e != cudaSuccess) return e;
+        chunk_state_kernel<__nv_bfloat16><<<gc, kThreads, ss, st>>>(
+            plan, d, static_cast<const __nv_bfloat16 *>(a.x), static_cast<const __nv_bfloat16 *>(a.B), a.cs, a.dv,
+            a.states);
+    } else {
+        chunk_cumsum_kernel<float><<<gc, d.Q, 0, st>>>(plan, d, static_cast<const float *>(a.dt), a.A_log, a.cs,
+                                                       a.dv);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(chunk_state_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ss);
+        if (e != cudaSuccess) return e;
+        chunk_state_kernel<float><<<gc, kThreads, ss, st>>>(plan, d, static_cast<const float *>(a.x),
+                                                            static_cast<const float *>(a.B), a.cs, a.dv, a.states);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const dim3 gp(plan.nseq, d.H, (d.P * d.N + kThreads - 1) / kThreads);
+    state_passing_kernel<<<gp, kThreads, 0, st>>>(plan, d, a.cs, a.states, a.init, nullptr);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_simt(const Plan &plan, const Dims &d, const SimtArgs &a, cudaStream_t stream,
                         const Instr &ins)

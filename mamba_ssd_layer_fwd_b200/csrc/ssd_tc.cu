@@ -18,6 +18,10 @@
 //                                          (state warps rescale H in TMEM, UMMA accumulates)
 //                                          Sec. 6.2 right + centre factors
 //
+// Exponents that are <= 0 in exact arithmetic (cs_l - cs_s with s <= l) are
+// clamped at 0: with a huge decay rate the fp32 prefix sums can round them
+// above 0, and the exponential would overflow.
+//
 // Each diagonal block of the caller's chunk length Q (128 or 256) is thereby
 // computed by the same decomposition one level down with 128-token blocks;
 // Sec. 6.1 leaves the method for a diagonal block free, and the result is
@@ -353,7 +357,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                 const float csn = excl + pre[i];
                 c2v[i] = csn * kLog2e;
                 // decay from token s to the block end (and, walking backwards, on to the segment end)
-                wv[i] = ex2_approx((STATE_ONLY ? last - csn + rs : last - csn) * kLog2e) * dl[i];
+                wv[i] = ex2_approx(fminf(STATE_ONLY ? last - csn + rs : last - csn, 0.0f) * kLog2e) * dl[i];
                 ev[i] = ex2_approx(c2v[i]);
             }
             // factorised mask: exp2(cs2_l - cs2_s) = exp2(cs2_l - R) * exp2(R - cs2_s) with R the
@@ -716,7 +720,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                             if (!exact) {
                                 // exp2(cs2_l - cs2_s) delta_s = exp2(cs2_l - R) * [exp2(R - cs2_s) delta_s]:
                                 // CB times the column factor, then the row factor of each 16-column chunk
-                                const float v0 = ex2_approx(rowc - R0), v1 = ex2_approx(rowc - R1);
+                                const float v0 = ex2_approx(fminf(rowc - R0, 0.0f)), v1 = ex2_approx(fminf(rowc - R1, 0.0f));
 #pragma unroll
                                 for (int i = 0; i < 32; i += 2)
                                     mul_f32x2(m[i], m[i + 1], __uint_as_float(r[i]), __uint_as_float(r[i + 1]), cf[i],
@@ -732,10 +736,10 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
 #pragma unroll
                                 for (int i4 = 0; i4 < 8; ++i4) {
                                     const float4 c4 = cc[i4], d4 = dd[i4];
-                                    m[4 * i4 + 0] = __uint_as_float(r[4 * i4 + 0]) * (ex2_approx(rowc - c4.x) * d4.x);
-                                    m[4 * i4 + 1] = __uint_as_float(r[4 * i4 + 1]) * (ex2_approx(rowc - c4.y) * d4.y);
-                                    m[4 * i4 + 2] = __uint_as_float(r[4 * i4 + 2]) * (ex2_approx(rowc - c4.z) * d4.z);
-                                    m[4 * i4 + 3] = __uint_as_float(r[4 * i4 + 3]) * (ex2_approx(rowc - c4.w) * d4.w);
+                                    m[4 * i4 + 0] = __uint_as_float(r[4 * i4 + 0]) * (ex2_approx(fminf(rowc - c4.x, 0.0f)) * d4.x);
+                                    m[4 * i4 + 1] = __uint_as_float(r[4 * i4 + 1]) * (ex2_approx(fminf(rowc - c4.y, 0.0f)) * d4.y);
+                                    m[4 * i4 + 2] = __uint_as_float(r[4 * i4 + 2]) * (ex2_approx(fminf(rowc - c4.z, 0.0f)) * d4.z);
+                                    m[4 * i4 + 3] = __uint_as_float(r[4 * i4 + 3]) * (ex2_approx(fminf(rowc - c4.w, 0.0f)) * d4.w);
                                 }
                             }
                             // pairs are 32-aligned like the warp's rows: only the pair holding the
