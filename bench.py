@@ -486,6 +486,10 @@ def run_ours(args):
             del sfw
             torch.cuda.empty_cache()
 
+    backward = None
+    if world == 1 and not args.no_sub_workloads:
+        backward = measure_backward(ssd, args, dev, flush)
+
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
@@ -510,12 +514,83 @@ def run_ours(args):
                                                      args.path)),
             "wall_s_timed_region": wall,
             "workloads": subs,
+            "backward": backward,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def backward_bytes(inp: dict) -> int:
+    """Compulsory traffic of one backward: x, dt, B, C, dy read (io dtype),
+    dx, ddt, dB, dC written (fp32), states read / gradients written."""
+    x, dt, B = inp["x"], inp["dt"], inp["B"]
+    es = 2 if inp["io_dtype"] == "bf16" else 4
+    n = (2 * x.size + dt.size + 2 * B.size) * es + (x.size + dt.size + 2 * B.size) * 4
+    H, P, N = x.shape[2], x.shape[3], B.shape[3]
+    nseq = inp["workload"].nseq
+    if inp.get("initial_states") is not None:
+        n += 2 * nseq * H * P * N * 4
+    return int(n)
+
+
+def measure_backward(ssd, args, dev, flush, steps=10):
+    """ssd_bwd on the headline workload after the timed forward region:
+    median device time of `steps` calls (L2 flushed before each), the output
+    checked against the gradient oracle on one sampled sequence."""
+    import torch
+    import oracle
+    inp = make_workload(args)
+    if inp["io_dtype"] != "bf16":
+        return None
+    host, d = _device_inputs(inp, dev)
+    rng = np.random.default_rng(1)
+    dy = ssd_inputs.round_to_bf16(rng.standard_normal(inp["x"].shape).astype(np.float32))
+    dy_t = torch.from_numpy(dy).to(dev, torch.bfloat16)
+    stream = torch.cuda.current_stream()
+
+    def run():
+        return ssd.ssd_bwd(d["x"], d["dt"], d["A_log"], d["B"], d["C"], d["D"], dy_t,
+                           initial_states=d["initial_states"], cu_seqlens=d["cu_seqlens"], stream=stream)
+
+    for _ in range(2):
+        flush.zero_()
+        g = run()
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g = run()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    # check one sequence (all its heads) against the gradient oracle
+    bounds = ssd_inputs.seq_bounds(inp)
+    t0, n = bounds[0]
+    one = dict(inp, x=inp["x"].reshape(-1, *inp["x"].shape[2:])[t0:t0 + n][None],
+               dt=inp["dt"].reshape(-1, inp["dt"].shape[2])[t0:t0 + n][None],
+               B=inp["B"].reshape(-1, *inp["B"].shape[2:])[t0:t0 + n][None],
+               C=inp["C"].reshape(-1, *inp["C"].shape[2:])[t0:t0 + n][None],
+               initial_states=None if inp["initial_states"] is None else inp["initial_states"][:1],
+               cu_seqlens=None)
+    want = oracle.recurrence_grad(one, dy.reshape(-1, *dy.shape[2:])[t0:t0 + n][None])
+    errs = {}
+    for k, kw in (("dx", "dx"), ("ddt", "ddt"), ("dB", "dB"), ("dC", "dC")):
+        got = g[k].reshape(-1, *g[k].shape[2:])[t0:t0 + n].double().cpu().numpy()
+        w = want[kw][0]
+        errs[k] = float(np.abs(got - w).max() / max(np.abs(w).max(), 1e-30))
+    tokens = inp["x"].shape[0] * inp["x"].shape[1]
+    med = statistics.median(ms)
+    nb = backward_bytes(inp)
+    peak, _ = measured_peaks()
+    return {"workload": inp["workload"].name, "ms": _stats(ms), "tokens_per_s": tokens / (med * 1e-3),
+            "alg_bytes": nb, "frac_hbm": nb / (med * 1e-3) / 1e9 / peak, "path": "simt (CUDA cores, fp32)",
+            "check": {"sequence": 0, "max_rel_err": errs, "tol": 1e-3,
+                      "ok": bool(max(errs.values()) <= 1e-3)}}
 
 
 def fw_launches(ssd, inp, path):

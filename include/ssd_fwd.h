@@ -207,6 +207,45 @@ SSD_API ssd_status ssd_decode_step(const ssd_step_params *p,
                    const void *B, const void *C, const float *D,
                    float *state, void *y, void *stream);
 
+/* Context parallelism ("Transformers are SSMs", Sec. 8.2 item 2, Fig. 7
+ * right): a long sequence is cut into pieces held by different workers; a
+ * worker takes the state entering its piece, runs the SSM on it and passes
+ * its final state on.  Since a piece maps an entering state H to
+ * exp(L) H + S, with S its end state from a zero state and L its total log
+ * decay (sum over its tokens of delta_t * A), the workers can summarise their
+ * pieces at the same time, exchange the summaries once, and each fold the
+ * summaries of the pieces before its own:
+ *
+ *   1. ssd_fwd_summary on the local piece          -> S (nseq, nheads, headdim, dstate), L (nseq, nheads)
+ *   2. all-gather S and L over the workers         (the caller's collective, e.g. NCCL)
+ *   3. ssd_state_combine(world, rank, ...)         -> the state entering this piece
+ *   4. ssd_fwd on the local piece from that state  -> y of the piece (and, on the last worker, the
+ *                                                     final state)
+ *
+ * ssd_fwd_summary takes ssd_fwd's parameters and inputs (C and D are not
+ * needed) and writes, for every sequence of the call, its end state from a
+ * zero state (end_states, float32) and its total log decay (logdecay,
+ * float32, (nseq, nheads)).  Its workspace is ssd_fwd's
+ * (ssd_fwd_summary_workspace_size).  Errors and asynchrony as for ssd_fwd.
+ *
+ * ssd_state_combine folds the summaries of workers 0 .. rank-1, in order,
+ * starting from initial_states (NULL = 0): H <- exp(L_r) H + S_r.
+ * end_states_all is (world, nseq, nheads, headdim, dstate) and logdecay_all
+ * (world, nseq, nheads), float32 device arrays; entering_states receives
+ * (nseq, nheads, headdim, dstate).  rank == world gives the state after the
+ * whole sequence.  Returns SSD_ERR_INVALID_ARG for a bad size or NULL array,
+ * SSD_ERR_CUDA if the launch fails. */
+SSD_API size_t ssd_fwd_summary_workspace_size(const ssd_fwd_params *p);
+
+SSD_API ssd_status ssd_fwd_summary(const ssd_fwd_params *p,
+                   const void *x, const void *dt, const float *A_log, const void *B,
+                   const int32_t *cu_seqlens, float *end_states, float *logdecay,
+                   void *workspace, size_t workspace_bytes, void *stream);
+
+SSD_API ssd_status ssd_state_combine(int world, int rank, int nseq, int nheads, int headdim, int dstate,
+                   const float *end_states_all, const float *logdecay_all,
+                   const float *initial_states, float *entering_states, void *stream);
+
 /* Backward pass: the gradients of a loss L given dy = dL/dy and
  * dfinal_states = dL/dfinal_states, for training ("Transformers are SSMs",
  * Thm. 6.1 counts the training cost of the SSD algorithm; the gradient is the

@@ -22,7 +22,7 @@ import threading
 from typing import Optional
 
 __all__ = [
-    "ssd_fwd", "ssd_bwd", "ssd_decode_step", "SsdParams", "SsdStepParams", "SsdInstrumentation", "make_instrumentation", "workspace_size",
+    "ssd_fwd", "ssd_bwd", "ssd_fwd_summary", "ssd_state_combine", "ssd_decode_step", "SsdParams", "SsdStepParams", "SsdInstrumentation", "make_instrumentation", "workspace_size",
     "launch_count", "resolved_path", "library", "library_path", "STATUS", "PATHS", "SsdError",
 ]
 
@@ -36,7 +36,8 @@ STATUS = {0: "SSD_OK", -1: "SSD_ERR_INVALID_ARG", -2: "SSD_ERR_UNSUPPORTED", -3:
 PATHS = {"auto": 0, "simt": 1, "tensor": 2}
 DTYPES = {"f32": 0, "bf16": 1}
 
-EXPORTED = ("ssd_fwd", "ssd_fwd_instrumented", "ssd_bwd", "ssd_bwd_workspace_size", "ssd_decode_step", "ssd_fwd_workspace_size", "ssd_get_status", "ssd_fwd_launch_count",
+EXPORTED = ("ssd_fwd", "ssd_fwd_instrumented", "ssd_bwd", "ssd_bwd_workspace_size", "ssd_fwd_summary",
+            "ssd_fwd_summary_workspace_size", "ssd_state_combine", "ssd_decode_step", "ssd_fwd_workspace_size", "ssd_get_status", "ssd_fwd_launch_count",
             "ssd_fwd_resolved_path", "ssd_status_string", "ssd_abi_version")
 
 
@@ -95,6 +96,12 @@ def library():
             lib.ssd_bwd.argtypes = [pp] + [vp] * 17 + [vp, sz, vp]
             lib.ssd_bwd_workspace_size.restype = sz
             lib.ssd_bwd_workspace_size.argtypes = [pp]
+            lib.ssd_fwd_summary.restype = i32
+            lib.ssd_fwd_summary.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+            lib.ssd_fwd_summary_workspace_size.restype = sz
+            lib.ssd_fwd_summary_workspace_size.argtypes = [pp]
+            lib.ssd_state_combine.restype = i32
+            lib.ssd_state_combine.argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp]
             lib.ssd_decode_step.restype = i32
             lib.ssd_decode_step.argtypes = [ctypes.POINTER(SsdStepParams), vp, vp, vp, vp, vp, vp, vp, vp, vp]
             lib.ssd_fwd_workspace_size.restype = sz
@@ -233,6 +240,64 @@ def ssd_fwd(x, dt, A_log, B, C, D=None, chunk_len: int = 256, initial_states=Non
         if rc != 0:
             raise SsdError(rc, "ssd_fwd (device status)")
     return (y, final_states) if want_final else y
+
+
+def ssd_fwd_summary(x, dt, A_log, B, chunk_len: int = 256, cu_seqlens=None, dt_softplus: bool = True,
+                    path: str = "auto", workspace=None, stream=None, check_status: bool = False):
+    """Every sequence's end state from a zero state, (nseq, H, P, N) float32,
+    and its total log decay sum_t delta_t A, (nseq, H) float32, through the
+    C ABI (the summary one worker of a context-parallel forward exchanges)."""
+    import torch
+    lib = library()
+    dev = x.device
+    if dev.type != "cuda":
+        raise ValueError("ssd_fwd_summary runs on CUDA tensors only")
+    for name, t in (("x", x), ("dt", dt), ("B", B)):
+        if t.dtype != x.dtype or not t.is_contiguous() or t.device != dev:
+            raise ValueError(f"{name} must be a contiguous {x.dtype} tensor on {dev}")
+    p = params_for(x, B, chunk_len, cu_seqlens, dt_softplus, path)
+    b, T, H, P = x.shape
+    N = B.shape[3]
+    nseq = p.num_seqs if p.num_seqs > 0 else b
+    S = torch.empty((nseq, H, P, N), dtype=torch.float32, device=dev)
+    L = torch.empty((nseq, H), dtype=torch.float32, device=dev)
+    need = int(lib.ssd_fwd_summary_workspace_size(ctypes.byref(p)))
+    if need == 0:
+        raise SsdError(-2 if lib.ssd_fwd_resolved_path(ctypes.byref(p)) == -1 else -1, "ssd_fwd_summary_workspace_size")
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    st = _stream_handle(stream)
+    rc = lib.ssd_fwd_summary(ctypes.byref(p), _ptr(x), _ptr(dt), _ptr(A_log), _ptr(B), _ptr(cu_seqlens), _ptr(S),
+                             _ptr(L), _ptr(workspace), workspace.numel() * workspace.element_size(), st)
+    if rc != 0:
+        raise SsdError(rc, "ssd_fwd_summary")
+    if check_status:
+        rc = lib.ssd_get_status(_ptr(workspace), st)
+        if rc != 0:
+            raise SsdError(rc, "ssd_fwd_summary (device status)")
+    return S, L
+
+
+def ssd_state_combine(end_states_all, logdecay_all, rank: int, initial_states=None, out=None, stream=None):
+    """Fold the summaries of workers 0 .. rank-1 (end_states_all (world, nseq,
+    H, P, N), logdecay_all (world, nseq, H), float32) from initial_states:
+    the state entering worker `rank` (rank == world: after the last piece)."""
+    import torch
+    lib = library()
+    world, nseq, H, P, N = end_states_all.shape
+    for name, t in (("end_states_all", end_states_all), ("logdecay_all", logdecay_all),
+                    ("initial_states", initial_states)):
+        if t is not None and (t.dtype != torch.float32 or not t.is_contiguous() or t.device.type != "cuda"):
+            raise ValueError(f"{name} must be a contiguous float32 CUDA tensor")
+    if tuple(logdecay_all.shape) != (world, nseq, H):
+        raise ValueError("logdecay_all must be (world, nseq, nheads)")
+    if out is None:
+        out = torch.empty((nseq, H, P, N), dtype=torch.float32, device=end_states_all.device)
+    rc = lib.ssd_state_combine(int(world), int(rank), int(nseq), int(H), int(P), int(N), _ptr(end_states_all),
+                               _ptr(logdecay_all), _ptr(initial_states), _ptr(out), _stream_handle(stream))
+    if rc != 0:
+        raise SsdError(rc, "ssd_state_combine")
+    return out
 
 
 def ssd_bwd(x, dt, A_log, B, C, D, dy, initial_states=None, cu_seqlens=None, dfinal_states=None,

@@ -223,6 +223,91 @@ ssd_status ssd_fwd_instrumented(const ssd_fwd_params *p, const void *x, const vo
     }
 }
 
+size_t ssd_fwd_summary_workspace_size(const ssd_fwd_params *p)
+{
+    return ssd_fwd_workspace_size(p);
+}
+
+ssd_status ssd_fwd_summary(const ssd_fwd_params *p, const void *x, const void *dt, const float *A_log, const void *B,
+                           const int32_t *cu_seqlens, float *end_states, float *logdecay, void *workspace,
+                           size_t workspace_bytes, void *stream)
+{
+    try {
+        const ssd_status v = validate(p);
+        if (v != SSD_OK) return v;
+        const bool has_tokens = (long long)p->batch * p->seqlen > 0;
+        if (!A_log || !workspace || !end_states || !logdecay) return SSD_ERR_INVALID_ARG;
+        if (has_tokens && (!x || !dt || !B)) return SSD_ERR_INVALID_ARG;
+        if ((p->num_seqs > 0) != (cu_seqlens != nullptr)) return SSD_ERR_INVALID_ARG;
+        const void *ptrs[] = {x, dt, A_log, B, cu_seqlens, end_states, logdecay};
+        for (const void *q : ptrs)
+            if (q && !aligned16(q)) return SSD_ERR_INVALID_ARG;
+        if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0) return SSD_ERR_INVALID_ARG;
+        const int path = resolve_path(*p);
+        if (path < 0) return SSD_ERR_UNSUPPORTED;
+        const Layout L = layout_of(*p, path);
+        if (workspace_bytes < L.total) return SSD_ERR_INVALID_ARG;
+        cudaStream_t st = static_cast<cudaStream_t>(stream);
+        char *ws = static_cast<char *>(workspace);
+        Plan plan;
+        plan.status = reinterpret_cast<int *>(ws + L.status);
+        plan.count = reinterpret_cast<int *>(ws + L.count);
+        plan.chunks = reinterpret_cast<ChunkDesc *>(ws + L.chunks);
+        plan.seqs = reinterpret_cast<SeqDesc *>(ws + L.seqs);
+        plan.nseq = nseq_of(*p);
+        plan.max_chunks = max_chunks_of(*p);
+        cudaError_t e;
+        if (path == SSD_PATH_SIMT) {
+            Dims d;
+            d.H = p->nheads;
+            d.P = p->headdim;
+            d.N = p->dstate;
+            d.G = p->ngroups;
+            d.Q = p->chunk_len;
+            d.heads_per_group = p->nheads / p->ngroups;
+            d.tokens = p->batch * p->seqlen;
+            d.dt_softplus = p->dt_softplus;
+            if (launch_build_plan(plan, cu_seqlens, p->batch, p->seqlen, p->chunk_len, st) != cudaSuccess)
+                return SSD_ERR_CUDA;
+            SimtArgs a;
+            a.x = x; a.dt = dt; a.B = B; a.C = nullptr;
+            a.A_log = A_log; a.D = nullptr; a.init = nullptr;
+            a.y = nullptr; a.final_states = nullptr;
+            a.cs = reinterpret_cast<float *>(ws + L.cs);
+            a.dv = reinterpret_cast<float *>(ws + L.dv);
+            a.states = reinterpret_cast<float *>(ws + L.states);
+            a.bf16 = p->io_dtype == SSD_DTYPE_BF16;
+            e = launch_simt_summary(plan, d, a, end_states, logdecay, st);
+        } else {
+            TcArgs a;
+            a.x = x; a.dt = dt; a.B = B; a.C = nullptr;
+            a.A_log = A_log; a.D = nullptr; a.init = nullptr;
+            a.cu_seqlens = cu_seqlens;
+            a.y = nullptr; a.final_states = nullptr;
+            a.scratch = ws + L.tc;
+            a.scratch_bytes = L.total - L.tc;
+            e = launch_tc_summary(*p, plan, a, end_states, logdecay, st);
+        }
+        return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+    } catch (...) {
+        return SSD_ERR_CUDA;
+    }
+}
+
+ssd_status ssd_state_combine(int world, int rank, int nseq, int nheads, int headdim, int dstate,
+                             const float *end_states_all, const float *logdecay_all, const float *initial_states,
+                             float *entering_states, void *stream)
+{
+    if (world < 1 || rank < 0 || rank > world || nseq < 0 || nheads < 1 || headdim < 1 || dstate < 1)
+        return SSD_ERR_INVALID_ARG;
+    if (!end_states_all || !logdecay_all || !entering_states) return SSD_ERR_INVALID_ARG;
+    const long long nsh = (long long)nseq * nheads;
+    if (nsh * headdim * dstate * (long long)world >= (1LL << 40)) return SSD_ERR_UNSUPPORTED;
+    const cudaError_t e = launch_state_combine(world, rank, nsh, headdim * dstate, end_states_all, logdecay_all,
+                                               initial_states, entering_states, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
 namespace {
 
 struct BwdLayout {

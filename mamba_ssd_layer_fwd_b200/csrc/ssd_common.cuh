@@ -98,6 +98,10 @@ struct SimtArgs {
 };
 cudaError_t launch_simt(const Plan &plan, const Dims &d, const SimtArgs &a, cudaStream_t stream,
                         const Instr &ins);
+// Ordered fold of per-worker state summaries (ssd_cp.cu).
+cudaError_t launch_state_combine(int world, int rank, long long nsh, int PN, const float *S_all, const float *L_all,
+                                 const float *init, float *H_in, cudaStream_t st);
+
 // Backward pass (ssd_bwd.cu): 32-token chunks, fp32 gradients.
 bool bwd_supported(const ssd_fwd_params &p);
 size_t bwd_chunk_count(const ssd_fwd_params &p);
@@ -108,6 +112,11 @@ cudaError_t launch_bwd(const Plan &plan, const Dims &d, const SimtArgs &fa, cons
 
 // The first three SIMT kernels only (chunk cumsum, chunk states, state
 // passing): cs, dv and, in `states`, the state entering every chunk.
-cudaError_t launch_simt_states(const Plan &plan, const Dims &d, const SimtArgs &a, cudaStream_t stream);
+cudaError_t launch_simt_states(const Plan &plan, const Dims &d, const SimtArgs &a, cudaStream_t stream,
+                               float *final_states = nullptr);
+// Every sequence's end state from a zero state and its total log decay
+// sum_t delta_t A (SIMT kernels).
+cudaError_t launch_simt_summary(const Plan &plan, const Dims &d, const SimtArgs &a, float *end_states,
+                                float *logdecay, cudaStream_t stream);
 
 }  // namespace ssd

@@ -314,9 +314,24 @@ cudaError_t launch_typed(const Plan &plan, const Dims &d, const SimtArgs &a, cud
     return cudaGetLastError();
 }
 
+// Total log decay sum_t delta_t A of every (sequence, head): the sum of its
+// chunks' last prefix sums.
+__global__ void __launch_bounds__(kThreads)
+seq_logdecay_kernel(Plan plan, Dims d, const float *__restrict__ cs, float *__restrict__ logdecay)
+{
+    const int i = blockIdx.x * kThreads + threadIdx.x;
+    if (i >= plan.nseq * d.H) return;
+    const int s = i / d.H, h = i % d.H;
+    const SeqDesc sq = plan.seqs[s];
+    float v = 0.0f;
+    for (int j = 0; j < sq.nchunks; ++j) v += cs[((size_t)(sq.chunk0 + j) * d.H + h) * d.Q + d.Q - 1];
+    logdecay[i] = v;
+}
+
 }  // namespace
 
-cudaError_t launch_simt_states(const Plan &plan, const Dims &d, const SimtArgs &a, cudaStream_t st)
+cudaError_t launch_simt_states(const Plan &plan, const Dims &d, const SimtArgs &a, cudaStream_t st,
+                               float *final_states)
 {
     if (plan.max_chunks == 0) return cudaSuccess;
     const dim3 gc(plan.max_chunks, d.H);
@@ -343,7 +358,24 @@ cudaError_t launch_simt_states(const Plan &plan, const Dims &d, const SimtArgs &
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const dim3 gp(plan.nseq, d.H, (d.P * d.N + kThreads - 1) / kThreads);
-    state_passing_kernel<<<gp, kThreads, 0, st>>>(plan, d, a.cs, a.states, a.init, nullptr);
+    state_passing_kernel<<<gp, kThreads, 0, st>>>(plan, d, a.cs, a.states, a.init, final_states);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_simt_summary(const Plan &plan, const Dims &d, const SimtArgs &a, float *end_states,
+                                float *logdecay, cudaStream_t st)
+{
+    cudaError_t e = launch_simt_states(plan, d, a, st, end_states);
+    if (e != cudaSuccess) return e;
+    if (plan.max_chunks == 0) {
+        // no tokens: zero end states (no initial state is applied in a summary)
+        const dim3 gp(plan.nseq, d.H, (d.P * d.N + kThreads - 1) / kThreads);
+        if (plan.nseq > 0)
+            state_passing_kernel<<<gp, kThreads, 0, st>>>(plan, d, a.cs, a.states, nullptr, end_states);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    const int n = plan.nseq * d.H;
+    if (n > 0) seq_logdecay_kernel<<<(n + kThreads - 1) / kThreads, kThreads, 0, st>>>(plan, d, a.cs, logdecay);
     return cudaGetLastError();
 }
 

@@ -91,6 +91,8 @@ struct TcParams {
     int H, G, N, heads_per_group;
     int dt_softplus;
     int withhold_x0;      // testing: work item 0 never loads its first x tile (bounded waits expire)
+    int summary;          // state-only mode over whole sequences: end state from zero and total
+                          // log decay of every sequence, written to row `seq` of segstate / seglogdec
 };
 
 // softplus(v) = max(v, 0) + log1p(e), e = exp(-|v|) in (0, 1], in a dozen
@@ -205,7 +207,8 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
         it.h0 = g0 - row * prm.H;
         it.pad = 0;
     }
-    if (STATE_ONLY && it.seg >= it.nseg - 1) return;   // only non-final segments need end states
+    // only non-final segments need end states (every sequence's, for a summary)
+    if (STATE_ONLY && !prm.summary && it.seg >= it.nseg - 1) return;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q = warp & 3;                             // SM sub-partition = TMEM lane quarter
@@ -1048,7 +1051,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                 const int h = it.h0 + j;
                 float *dst = nullptr;
                 if (STATE_ONLY)
-                    dst = prm.segstate + ((size_t)it.gseg * prm.H + h) * PN;
+                    dst = prm.segstate + ((size_t)(prm.summary ? it.seq : it.gseg) * prm.H + h) * PN;
                 else if (it.seg == it.nseg - 1 && prm.final_states)
                     dst = prm.final_states + ((size_t)it.seq * prm.H + h) * PN;
 #pragma unroll
@@ -1066,7 +1069,8 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                         }
                     }
                 }
-                if (STATE_ONLY && t == 0) prm.seglogdec[(size_t)it.gseg * prm.H + h] = ldec_sum[j];
+                if (STATE_ONLY && t == 0)
+                    prm.seglogdec[(size_t)(prm.summary ? it.seq : it.gseg) * prm.H + h] = ldec_sum[j];
             }
         }
         if (kTmaY && lane == 0) bulk_wait_all();       // this warp's y stores have landed
@@ -1482,6 +1486,7 @@ cudaError_t launch_tc(const ssd_fwd_params &p, const Plan &plan, const Dims &d, 
     prm.heads_per_group = d.heads_per_group;
     prm.dt_softplus = p.dt_softplus;
     prm.withhold_x0 = ins.withhold_first_tile != 0;
+    prm.summary = 0;
 
     if (ins.begin) cudaEventRecord(ins.begin, stream);
     if (s.segmented) {
@@ -1508,6 +1513,66 @@ cudaError_t launch_tc(const ssd_fwd_params &p, const Plan &plan, const Dims &d, 
     }
     if (ins.end) cudaEventRecord(ins.end, stream);
     return e;
+}
+
+// State summary on the tensor-core path: every sequence's end state from a
+// zero state and its total log decay, by the state-only walk over whole
+// sequences (one segment each).
+cudaError_t launch_tc_summary(const ssd_fwd_params &p, const Plan &plan, const TcArgs &a, float *end_states,
+                              float *logdecay, cudaStream_t stream)
+{
+    TcPlanShape s = plan_shape(p);
+    const long long tokens = (long long)p.batch * p.seqlen;
+    const int nseq = plan.nseq;
+    s.seg_len = (int)(p.num_seqs > 0 ? (tokens > 0 ? tokens : 1) : (p.seqlen > 0 ? p.seqlen : 1));
+    s.max_segments = nseq;
+    s.max_items = nseq * s.n_hb;
+    s.segmented = false;
+    TcItem *items = reinterpret_cast<TcItem *>(a.scratch);
+    const int PN = kP * p.dstate;
+    cudaError_t e = cudaMemsetAsync(logdecay, 0, sizeof(float) * (size_t)nseq * p.nheads, stream);
+    if (e != cudaSuccess) return e;
+    const bool direct = p.num_seqs == 0;
+    if (direct) {
+        e = cudaMemsetAsync(plan.status, 0, sizeof(int), stream);
+    } else {
+        // empty sequences get a zero end state here (no initial state); the others get items
+        tc_plan_kernel<<<1, 1024, 0, stream>>>(a.cu_seqlens, nseq, p.seqlen, s.seg_len, s.n_hb, s.KH, items,
+                                               plan.count, s.max_items, plan.status, nullptr, end_states,
+                                               p.nheads, PN, nullptr);
+        e = cudaGetLastError();
+    }
+    if (e != cudaSuccess || tokens == 0) return e;
+    CUtensorMap mX, mB;
+    if (!make_map(&mX, a.x, (uint64_t)p.nheads * kP, (uint64_t)tokens) ||
+        !make_map(&mB, a.B, (uint64_t)p.ngroups * p.dstate, (uint64_t)tokens))
+        return cudaErrorInvalidValue;
+    TcParams prm{};
+    prm.dt = static_cast<const __nv_bfloat16 *>(a.dt);
+    prm.A_log = a.A_log;
+    prm.segstate = end_states;
+    prm.seglogdec = logdecay;
+    prm.items = direct ? nullptr : items;
+    prm.count = plan.count;
+    prm.n_items = s.max_items;
+    prm.direct_base = 0;
+    prm.seqlen = p.seqlen;
+    prm.status = plan.status;
+    prm.H = p.nheads;
+    prm.G = p.ngroups;
+    prm.N = p.dstate;
+    prm.heads_per_group = p.nheads / p.ngroups;
+    prm.dt_softplus = p.dt_softplus;
+    prm.summary = 1;
+    // C and y maps are not read in state-only mode
+    return launch_walk_any<true>(p.dstate, s.KH, s.max_items, mX, mB, mB, mX, prm, stream);
+}
+
+size_t tc_summary_workspace_bytes(const ssd_fwd_params &p)
+{
+    const TcPlanShape s = plan_shape(p);
+    const int nseq = p.num_seqs > 0 ? p.num_seqs : p.batch;
+    return align256(sizeof(TcItem) * (size_t)nseq * s.n_hb);
 }
 
 }  // namespace ssd

@@ -20,5 +20,8 @@ size_t tc_workspace_bytes(const ssd_fwd_params &p);
 int tc_launch_count(const ssd_fwd_params &p);
 cudaError_t launch_tc(const ssd_fwd_params &p, const Plan &plan, const Dims &d, const TcArgs &a,
                       cudaStream_t stream, const Instr &ins);
+cudaError_t launch_tc_summary(const ssd_fwd_params &p, const Plan &plan, const TcArgs &a, float *end_states,
+                              float *logdecay, cudaStream_t stream);
+size_t tc_summary_workspace_bytes(const ssd_fwd_params &p);
 
 }  // namespace ssd
