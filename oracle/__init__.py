@@ -13,6 +13,8 @@ Structured State Space Duality":
   (sequence, head) pairs. This is the oracle the CUDA path is compared with.
 * `recurrence_grad` - reverse mode of the same recurrence (every input's
   gradient given dL/dy and dL/dfinal), plain C, fp64.
+* `gated_group_norm` - the block's output normalisation after the layer
+  (y * silu(z), then GroupNorm over each head's channels), numpy fp64.
 * `quadratic_form` - the dual (attention-like) mode, Sec. 3.4.2 / Sec. 5.1: build
   the T x T semiseparable matrix M[i, j] = C_i . (a_{j+1} ... a_i) B_j delta_j
   (lower triangle) explicitly and multiply. numpy, tiny sizes only. It pins the
@@ -190,6 +192,32 @@ def recurrence_grad(inp: dict, dy, dfinal=None, nthreads: int = 0) -> dict:
     out["dB"] = out["dB"].reshape(Bm.shape)
     out["dC"] = out["dC"].reshape(Cm.shape)
     return out
+
+
+def silu(z):
+    """z * sigmoid(z) in float64."""
+    z = np.asarray(z, dtype=np.float64)
+    return z / (1.0 + np.exp(-z))
+
+
+def gated_group_norm(y, z, weight, bias=None, eps: float = 1e-5, group_size=None):
+    """The Mamba-2 block's output normalisation ("Transformers are SSMs",
+    Sec. 7.1 extra normalisation before the output projection, Sec. 8.1
+    GroupNorm): g = y * silu(z), then every group of `group_size` consecutive
+    channels of a token (default: one head's headdim channels) is normalised
+    by its mean and variance, out = (g - mean) / sqrt(var + eps) * weight + bias.
+    y, z: (..., H, P); weight, bias: (H * P,). float64 result, y's shape."""
+    y = np.asarray(y, dtype=np.float64)
+    z = np.asarray(z, dtype=np.float64)
+    H, P = y.shape[-2], y.shape[-1]
+    gs = P if group_size is None else int(group_size)
+    g = (y * silu(z)).reshape(-1, H * P // gs, gs)
+    mean = g.mean(axis=-1, keepdims=True)
+    var = ((g - mean) ** 2).mean(axis=-1, keepdims=True)
+    out = ((g - mean) / np.sqrt(var + eps)).reshape(-1, H * P) * np.asarray(weight, dtype=np.float64)
+    if bias is not None:
+        out = out + np.asarray(bias, dtype=np.float64)
+    return out.reshape(y.shape)
 
 
 def _softplus(r):

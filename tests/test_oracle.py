@@ -448,3 +448,42 @@ def test_gradient_of_empty_sequence_passes_dfinal_through():
     dfin = rng.standard_normal(inp["initial_states"].shape).astype(np.float32)
     g = oracle.recurrence_grad(inp, dy, dfin)
     np.testing.assert_array_equal(g["dinit"][1], dfin[1].astype(np.float64))
+
+
+# ------------------------------------------------ gated norm of the Mamba-2 block
+
+def test_gated_group_norm_matches_torch_group_norm():
+    """Sec. 7.1 / 8.1: y * silu(z) followed by GroupNorm with one group per
+    head, against torch's own silu and group_norm (library routines, float64)."""
+    import torch
+    rng = np.random.default_rng(30)
+    T, H, P = 37, 6, 16
+    y = rng.standard_normal((T, H, P))
+    z = rng.standard_normal((T, H, P)) * 2.0
+    w = rng.standard_normal(H * P)
+    b = rng.standard_normal(H * P)
+    got = oracle.gated_group_norm(y, z, w, b, eps=1e-5)
+    g = torch.from_numpy(y) * torch.nn.functional.silu(torch.from_numpy(z))
+    want = torch.nn.functional.group_norm(g.reshape(T, H * P), H, torch.from_numpy(w), torch.from_numpy(b), 1e-5)
+    assert rel_err(got.reshape(T, H * P), want.numpy()) < 1e-12
+    # groups of 8 channels (two per head)
+    got8 = oracle.gated_group_norm(y, z, w, None, eps=1e-3, group_size=8)
+    want8 = torch.nn.functional.group_norm(g.reshape(T, H * P), H * P // 8, torch.from_numpy(w), None, 1e-3)
+    assert rel_err(got8.reshape(T, H * P), want8.numpy()) < 1e-12
+
+
+def test_gated_group_norm_closed_forms():
+    rng = np.random.default_rng(31)
+    T, H, P = 5, 3, 8
+    y = rng.standard_normal((T, H, P))
+    b = rng.standard_normal(H * P)
+    # z == 0 closes the gate: every group is constant 0, so the output is the bias
+    out = oracle.gated_group_norm(y, np.zeros_like(y), np.ones(H * P), b)
+    assert rel_err(out.reshape(T, H * P), np.broadcast_to(b, (T, H * P))) < 1e-15
+    # unit weight, no bias: every group has mean 0 and variance var / (var + eps)
+    z = rng.standard_normal((T, H, P))
+    out = oracle.gated_group_norm(y, z, np.ones(H * P), None, eps=1e-2).reshape(T, H, P)
+    g = y * z / (1 + np.exp(-z))
+    var = g.var(axis=-1)
+    assert np.max(np.abs(out.mean(axis=-1))) < 1e-14
+    assert rel_err(out.var(axis=-1), var / (var + 1e-2)) < 1e-12
