@@ -207,6 +207,28 @@ SSD_API ssd_status ssd_decode_step(const ssd_step_params *p,
                    const void *B, const void *C, const float *D,
                    float *state, void *y, void *stream);
 
+/* The SSD forward followed by the Mamba-2 block's output normalisation
+ * ("Transformers are SSMs", Sec. 7.1: an extra normalisation layer before the
+ * block's output projection; Sec. 8.1: a GroupNorm whose group count divides
+ * by the tensor-parallel degree), with the gate of the block's z branch:
+ *
+ *     g   = y * silu(z),   silu(z) = z / (1 + exp(-z))
+ *     out = (g - mean) / sqrt(var + eps) * norm_weight + norm_bias
+ *
+ * mean and var over each group of headdim channels of one token and head (one
+ * group per head).  z has y's layout and io dtype; norm_weight and norm_bias
+ * (NULL = 0) are float32 (nheads * headdim); out receives the normalised
+ * output in y's layout (y itself is not written).  The tensor-core path fuses
+ * the gate and the norm into its output epilogue; the SIMT path runs them as
+ * one more pass over out.  Other arguments, limits, errors and the workspace
+ * are ssd_fwd's; eps must be >= 0. */
+SSD_API ssd_status ssd_fwd_gated_norm(const ssd_fwd_params *p,
+                   const void *x, const void *dt, const float *A_log,
+                   const void *B, const void *C, const float *D,
+                   const float *initial_states, const int32_t *cu_seqlens,
+                   const void *z, const float *norm_weight, const float *norm_bias, float eps,
+                   void *out, float *final_states, void *workspace, size_t workspace_bytes, void *stream);
+
 /* Context parallelism ("Transformers are SSMs", Sec. 8.2 item 2, Fig. 7
  * right): a long sequence is cut into pieces held by different workers; a
  * worker takes the state entering its piece, runs the SSM on it and passes

@@ -36,7 +36,7 @@ STATUS = {0: "SSD_OK", -1: "SSD_ERR_INVALID_ARG", -2: "SSD_ERR_UNSUPPORTED", -3:
 PATHS = {"auto": 0, "simt": 1, "tensor": 2}
 DTYPES = {"f32": 0, "bf16": 1}
 
-EXPORTED = ("ssd_fwd", "ssd_fwd_instrumented", "ssd_bwd", "ssd_bwd_workspace_size", "ssd_fwd_summary",
+EXPORTED = ("ssd_fwd", "ssd_fwd_instrumented", "ssd_fwd_gated_norm", "ssd_bwd", "ssd_bwd_workspace_size", "ssd_fwd_summary",
             "ssd_fwd_summary_workspace_size", "ssd_state_combine", "ssd_decode_step", "ssd_fwd_workspace_size", "ssd_get_status", "ssd_fwd_launch_count",
             "ssd_fwd_resolved_path", "ssd_status_string", "ssd_abi_version")
 
@@ -96,6 +96,8 @@ def library():
             lib.ssd_bwd.argtypes = [pp] + [vp] * 17 + [vp, sz, vp]
             lib.ssd_bwd_workspace_size.restype = sz
             lib.ssd_bwd_workspace_size.argtypes = [pp]
+            lib.ssd_fwd_gated_norm.restype = i32
+            lib.ssd_fwd_gated_norm.argtypes = [pp] + [vp] * 11 + [ctypes.c_float, vp, vp, vp, sz, vp]
             lib.ssd_fwd_summary.restype = i32
             lib.ssd_fwd_summary.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
             lib.ssd_fwd_summary_workspace_size.restype = sz
@@ -183,7 +185,8 @@ def params_for(x, B, chunk_len: int, cu_seqlens=None, dt_softplus=True, path="au
 def ssd_fwd(x, dt, A_log, B, C, D=None, chunk_len: int = 256, initial_states=None,
             cu_seqlens=None, dt_softplus: bool = True, return_final_states: bool = False,
             y=None, final_states=None, workspace=None, stream=None, path: str = "auto",
-            instrumentation: Optional[SsdInstrumentation] = None, check_status: bool = False):
+            instrumentation: Optional[SsdInstrumentation] = None, check_status: bool = False,
+            z=None, norm_weight=None, norm_bias=None, norm_eps: float = 1e-5):
     """SSD forward on the GPU through the C ABI. Returns y, or (y, final_states)
     when `return_final_states` is true (or `final_states` is given).
 
@@ -191,6 +194,10 @@ def ssd_fwd(x, dt, A_log, B, C, D=None, chunk_len: int = 256, initial_states=Non
     initial_states are float32; cu_seqlens is int32. Outputs and the workspace
     are allocated with torch on x's device unless passed in. `instrumentation`
     (make_instrumentation) routes the call through ssd_fwd_instrumented.
+    With `z` (x's layout and dtype) and `norm_weight` (float32, nheads * headdim)
+    the call returns the Mamba-2 block's normalised output instead of y:
+    GroupNorm(y * silu(z)) over each head's channels, times norm_weight, plus
+    norm_bias (ssd_fwd_gated_norm).
     """
     import torch
     lib = library()
@@ -229,7 +236,20 @@ def ssd_fwd(x, dt, A_log, B, C, D=None, chunk_len: int = 256, initial_states=Non
     args = (ctypes.byref(p), _ptr(x), _ptr(dt), _ptr(A_log), _ptr(B), _ptr(C), _ptr(D),
             _ptr(initial_states), _ptr(cu_seqlens), _ptr(y), _ptr(final_states),
             _ptr(workspace), workspace.numel() * workspace.element_size(), st)
-    if instrumentation is None:
+    if z is not None:
+        for name, t in (("z", z),):
+            if t.dtype != x.dtype or not t.is_contiguous() or t.shape != x.shape or t.device != dev:
+                raise ValueError(f"{name} must be a contiguous {x.dtype} tensor shaped like x")
+        for name, t in (("norm_weight", norm_weight), ("norm_bias", norm_bias)):
+            if t is not None and (t.dtype != torch.float32 or not t.is_contiguous() or t.numel() != H * P):
+                raise ValueError(f"{name} must be a contiguous float32 tensor of nheads * headdim values")
+        if norm_weight is None:
+            raise ValueError("norm_weight is required with z")
+        rc = lib.ssd_fwd_gated_norm(ctypes.byref(p), _ptr(x), _ptr(dt), _ptr(A_log), _ptr(B), _ptr(C), _ptr(D),
+                                    _ptr(initial_states), _ptr(cu_seqlens), _ptr(z), _ptr(norm_weight),
+                                    _ptr(norm_bias), float(norm_eps), _ptr(y), _ptr(final_states),
+                                    _ptr(workspace), workspace.numel() * workspace.element_size(), st)
+    elif instrumentation is None:
         rc = lib.ssd_fwd(*args)
     else:
         rc = lib.ssd_fwd_instrumented(*args, ctypes.byref(instrumentation))

@@ -143,10 +143,20 @@ ssd_status ssd_fwd(const ssd_fwd_params *p, const void *x, const void *dt, const
                                 workspace_bytes, stream, nullptr);
 }
 
-ssd_status ssd_fwd_instrumented(const ssd_fwd_params *p, const void *x, const void *dt, const float *A_log,
-                                const void *B, const void *C, const float *D, const float *initial_states,
-                                const int32_t *cu_seqlens, void *y, float *final_states, void *workspace,
-                                size_t workspace_bytes, void *stream, const ssd_fwd_instrumentation *instr)
+}  // extern "C"
+
+namespace {
+
+struct GnArgs {
+    const void *z;
+    const float *w, *b;
+    float eps;
+};
+
+ssd_status fwd_impl(const ssd_fwd_params *p, const void *x, const void *dt, const float *A_log, const void *B,
+                    const void *C, const float *D, const float *initial_states, const int32_t *cu_seqlens, void *y,
+                    float *final_states, void *workspace, size_t workspace_bytes, void *stream,
+                    const ssd_fwd_instrumentation *instr, const GnArgs *gn)
 {
     try {
         const ssd_status v = validate(p);
@@ -205,6 +215,9 @@ ssd_status ssd_fwd_instrumented(const ssd_fwd_params *p, const void *x, const vo
             a.states = reinterpret_cast<float *>(ws + L.states);
             a.bf16 = p->io_dtype == SSD_DTYPE_BF16;
             e = launch_simt(plan, d, a, st, ins);
+            if (e == cudaSuccess && gn)
+                e = launch_gated_norm((long long)d.tokens * d.H, d.H, d.P, a.bf16, y, gn->z, gn->w, gn->b, gn->eps,
+                                      st);
         } else {
             TcArgs a;
             a.x = x; a.dt = dt; a.B = B; a.C = C;
@@ -213,6 +226,12 @@ ssd_status ssd_fwd_instrumented(const ssd_fwd_params *p, const void *x, const vo
             a.y = y; a.final_states = final_states;
             a.scratch = ws + L.tc;
             a.scratch_bytes = L.total - L.tc;
+            if (gn) {
+                a.z = gn->z;
+                a.gn_w = gn->w;
+                a.gn_b = gn->b;
+                a.gn_eps = gn->eps;
+            }
             e = launch_tc(*p, plan, d, a, st, ins);
         }
         return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
@@ -221,6 +240,34 @@ ssd_status ssd_fwd_instrumented(const ssd_fwd_params *p, const void *x, const vo
     } catch (...) {
         return SSD_ERR_CUDA;
     }
+}
+
+}  // namespace
+
+extern "C" {
+
+ssd_status ssd_fwd_instrumented(const ssd_fwd_params *p, const void *x, const void *dt, const float *A_log,
+                                const void *B, const void *C, const float *D, const float *initial_states,
+                                const int32_t *cu_seqlens, void *y, float *final_states, void *workspace,
+                                size_t workspace_bytes, void *stream, const ssd_fwd_instrumentation *instr)
+{
+    return fwd_impl(p, x, dt, A_log, B, C, D, initial_states, cu_seqlens, y, final_states, workspace,
+                    workspace_bytes, stream, instr, nullptr);
+}
+
+ssd_status ssd_fwd_gated_norm(const ssd_fwd_params *p, const void *x, const void *dt, const float *A_log,
+                              const void *B, const void *C, const float *D, const float *initial_states,
+                              const int32_t *cu_seqlens, const void *z, const float *norm_weight,
+                              const float *norm_bias, float eps, void *out, float *final_states, void *workspace,
+                              size_t workspace_bytes, void *stream)
+{
+    if (!p || !norm_weight || !(eps >= 0.0f)) return SSD_ERR_INVALID_ARG;
+    if ((long long)p->batch * p->seqlen > 0 && !z) return SSD_ERR_INVALID_ARG;
+    if ((z && !aligned16(z)) || !aligned16(norm_weight) || (norm_bias && !aligned16(norm_bias)))
+        return SSD_ERR_INVALID_ARG;
+    const GnArgs gn{z, norm_weight, norm_bias, eps};
+    return fwd_impl(p, x, dt, A_log, B, C, D, initial_states, cu_seqlens, out, final_states, workspace,
+                    workspace_bytes, stream, nullptr, &gn);
 }
 
 size_t ssd_fwd_summary_workspace_size(const ssd_fwd_params *p)

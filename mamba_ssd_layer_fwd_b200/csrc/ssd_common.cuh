@@ -98,6 +98,10 @@ struct SimtArgs {
 };
 cudaError_t launch_simt(const Plan &plan, const Dims &d, const SimtArgs &a, cudaStream_t stream,
                         const Instr &ins);
+// Gated GroupNorm of the block output, in place on y (ssd_gnorm.cu).
+cudaError_t launch_gated_norm(long long rows, int H, int P, bool bf16, void *y, const void *z, const float *w,
+                              const float *b, float eps, cudaStream_t st);
+
 // Ordered fold of per-worker state summaries (ssd_cp.cu).
 cudaError_t launch_state_combine(int world, int rank, long long nsh, int PN, const float *S_all, const float *L_all,
                                  const float *init, float *H_in, cudaStream_t st);

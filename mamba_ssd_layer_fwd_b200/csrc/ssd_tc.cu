@@ -75,6 +75,15 @@ struct TcItem {
     int pad;
 };
 
+// Gated norm of the block output (walk variant GN): out = GroupNorm(y * silu(z))
+// over each head's 64 channels, with per-channel weight and bias.  A kernel
+// argument of its own, so that the other variants' parameter block is unchanged.
+struct GnParams {
+    const __nv_bfloat16 *z;
+    const float *w, *b;
+    float eps;
+};
+
 struct TcParams {
     const __nv_bfloat16 *dt;
     const float *A_log, *D, *init;
@@ -177,10 +186,11 @@ __device__ long long *g_trace = nullptr;
     } while (0)
 #endif
 
-template <int NST, int KH, bool STATE_ONLY>
+template <int NST, int KH, bool STATE_ONLY, bool GN = false>
 __global__ void __launch_bounds__(kThreadsTc, 1)
 ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapB,
-            const __grid_constant__ CUtensorMap mapC, const __grid_constant__ CUtensorMap mapY, const TcParams prm)
+            const __grid_constant__ CUtensorMap mapC, const __grid_constant__ CUtensorMap mapY, const TcParams prm,
+            const GnParams gnp)
 {
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment (128-byte swizzle atoms) computed as an offset from the
@@ -916,6 +926,80 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             const bool via_tma = kTmaY && valid == kQ;
             // the slot's w o X tile is free once the state UMMA of unit v has completed
             if (kTmaY && !mbar_wait<kInlW>(&S.xw_free[wi], (v / kXwD) & 1, abort)) return false;
+            if (GN) {
+                // Mamba-2 block output (Sec. 7.1): g = y * silu(z), staged as bf16 while the
+                // statistics accumulate (shifted by the row's first g), then normalised over the
+                // head's 64 channels with the per-channel weight and bias
+                const bool row_ok = via_tma || t < valid;
+                const __nv_bfloat16 *zrow = gnp.z + ((size_t)tok * prm.H + it.h0 + j) * kP;
+                float sh = 0.0f, s1 = 0.0f, s2 = 0.0f;
+#pragma unroll
+                for (int h0 = 0; h0 < kP; h0 += 32) {
+                    uint32_t yd[32];
+                    tmem_ld16(tb + lane_base + kColYd + h0, *reinterpret_cast<uint32_t(*)[16]>(&yd[0]));
+                    tmem_ld16(tb + lane_base + kColYd + h0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&yd[16]));
+                    tmem_ld_wait();
+                    if (h0 == kP - 32) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&S.yd_empty);
+                    }
+                    if (row_ok) {
+#pragma unroll
+                        for (int q8 = 0; q8 < 32; q8 += 8) {
+                            const uint4 zz = *reinterpret_cast<const uint4 *>(zrow + h0 + q8);
+                            const uint32_t zw[4] = {zz.x, zz.y, zz.z, zz.w};
+                            uint32_t pk[4];
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const int pp = q8 + 2 * i;
+                                float ya, yb;
+                                fma_f32x2(ya, yb, el, el, __uint_as_float(yo[h0 + pp]), __uint_as_float(yo[h0 + pp + 1]),
+                                          __uint_as_float(yd[pp]), __uint_as_float(yd[pp + 1]));
+                                const float2 zf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&zw[i]));
+                                const float ga = ya * __fdividef(zf.x, 1.0f + __expf(-zf.x));
+                                const float gb = yb * __fdividef(zf.y, 1.0f + __expf(-zf.y));
+                                if (h0 == 0 && pp == 0) sh = ga;
+                                const float da = ga - sh, db = gb - sh;
+                                s1 += da + db;
+                                s2 = fmaf(da, da, fmaf(db, db, s2));
+                                pk[i] = pack_bf16x2(ga, gb);
+                            }
+                            const uint4 v4 = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                            if (via_tma)
+                                *reinterpret_cast<uint4 *>(stage + sw128_offset(lane, h0 + q8)) = v4;
+                            else
+                                *reinterpret_cast<uint4 *>(dst + h0 + q8) = v4;
+                        }
+                    }
+                }
+                if (row_ok) {
+                    const float mo = s1 * (1.0f / kP);
+                    const float rstd = rsqrtf(fmaxf(s2 * (1.0f / kP) - mo * mo, 0.0f) + gnp.eps);
+                    const float mean = sh + mo;
+                    const float *wrow = gnp.w + (size_t)(it.h0 + j) * kP;
+                    const float *brow = gnp.b ? gnp.b + (size_t)(it.h0 + j) * kP : nullptr;
+#pragma unroll
+                    for (int c8 = 0; c8 < kP; c8 += 8) {
+                        uint4 *slot_ptr = via_tma ? reinterpret_cast<uint4 *>(stage + sw128_offset(lane, c8))
+                                                  : reinterpret_cast<uint4 *>(dst + c8);
+                        uint4 v4 = *slot_ptr;
+                        uint32_t *vw = reinterpret_cast<uint32_t *>(&v4);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float2 g2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&vw[i]));
+                            const int cc = c8 + 2 * i;
+                            float oa = (g2.x - mean) * rstd * wrow[cc], ob = (g2.y - mean) * rstd * wrow[cc + 1];
+                            if (brow) {
+                                oa += brow[cc];
+                                ob += brow[cc + 1];
+                            }
+                            vw[i] = pack_bf16x2(oa, ob);
+                        }
+                        *slot_ptr = v4;
+                    }
+                }
+            } else {
 #pragma unroll
             for (int h0 = 0; h0 < kP; h0 += 32) {
                 uint32_t yd[32];
@@ -946,6 +1030,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                             *reinterpret_cast<uint4 *>(dst + h0 + q8) = v4;
                     }
                 }
+            }
             }
             if (via_tma) fence_async_smem();
             __syncwarp();
@@ -1343,35 +1428,44 @@ TcPlanShape plan_shape(const ssd_fwd_params &p)
     return s;
 }
 
-template <int NST, int KH, bool SO>
+template <int NST, int KH, bool SO, bool GN>
 cudaError_t launch_walk(int grid, const CUtensorMap &mX, const CUtensorMap &mB, const CUtensorMap &mC,
                         const CUtensorMap &mY,
-                        const TcParams &prm, cudaStream_t st)
+                        const TcParams &prm, cudaStream_t st, const GnParams &gnp = GnParams{})
 {
     const size_t smem = tc_smem_bytes<NST>();
-    cudaError_t e = cudaFuncSetAttribute(ssd_tc_walk<NST, KH, SO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(ssd_tc_walk<NST, KH, SO, GN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    ssd_tc_walk<NST, KH, SO><<<grid, kThreadsTc, smem, st>>>(mX, mB, mC, mY, prm);
+    ssd_tc_walk<NST, KH, SO, GN><<<grid, kThreadsTc, smem, st>>>(mX, mB, mC, mY, prm, gnp);
     return cudaGetLastError();
 }
 
-template <int NST, bool SO>
+template <int NST, bool SO, bool GN>
 cudaError_t launch_walk_kh(int KH, int grid, const CUtensorMap &mX, const CUtensorMap &mB, const CUtensorMap &mC,
                            const CUtensorMap &mY,
-                           const TcParams &prm, cudaStream_t st)
+                           const TcParams &prm, cudaStream_t st, const GnParams &gnp = GnParams{})
 {
-    return KH == 2 ? launch_walk<NST, 2, SO>(grid, mX, mB, mC, mY, prm, st)
-                   : launch_walk<NST, 1, SO>(grid, mX, mB, mC, mY, prm, st);
+    return KH == 2 ? launch_walk<NST, 2, SO, GN>(grid, mX, mB, mC, mY, prm, st, gnp)
+                   : launch_walk<NST, 1, SO, GN>(grid, mX, mB, mC, mY, prm, st, gnp);
 }
 
-template <bool SO>
+template <bool SO, bool GN = false>
 cudaError_t launch_walk_any(int N, int KH, int grid, const CUtensorMap &mX, const CUtensorMap &mB,
-                            const CUtensorMap &mC, const CUtensorMap &mY, const TcParams &prm, cudaStream_t st)
+                            const CUtensorMap &mC, const CUtensorMap &mY, const TcParams &prm, cudaStream_t st,
+                            const GnParams &gnp = GnParams{})
 {
-    if (N == 256) return launch_walk_kh<256, SO>(KH, grid, mX, mB, mC, mY, prm, st);
-    return N == 128 ? launch_walk_kh<128, SO>(KH, grid, mX, mB, mC, mY, prm, st)
-                    : launch_walk_kh<64, SO>(KH, grid, mX, mB, mC, mY, prm, st);
+    if (N == 256) return launch_walk_kh<256, SO, GN>(KH, grid, mX, mB, mC, mY, prm, st, gnp);
+    return N == 128 ? launch_walk_kh<128, SO, GN>(KH, grid, mX, mB, mC, mY, prm, st, gnp)
+                    : launch_walk_kh<64, SO, GN>(KH, grid, mX, mB, mC, mY, prm, st, gnp);
+}
+
+// the output pass, with or without the gated norm epilogue
+cudaError_t launch_out(const GnParams &gnp, int N, int KH, int grid, const CUtensorMap &mX, const CUtensorMap &mB,
+                       const CUtensorMap &mC, const CUtensorMap &mY, const TcParams &prm, cudaStream_t st)
+{
+    return gnp.z ? launch_walk_any<false, true>(N, KH, grid, mX, mB, mC, mY, prm, st, gnp)
+                 : launch_walk_any<false, false>(N, KH, grid, mX, mB, mC, mY, prm, st);
 }
 
 size_t align256(size_t v) { return (v + 255) / 256 * 256; }
@@ -1487,6 +1581,7 @@ cudaError_t launch_tc(const ssd_fwd_params &p, const Plan &plan, const Dims &d, 
     prm.dt_softplus = p.dt_softplus;
     prm.withhold_x0 = ins.withhold_first_tile != 0;
     prm.summary = 0;
+    GnParams gnp{static_cast<const __nv_bfloat16 *>(a.z), a.gn_w, a.gn_b, a.gn_eps};
 
     if (ins.begin) cudaEventRecord(ins.begin, stream);
     if (s.segmented) {
@@ -1500,15 +1595,15 @@ cudaError_t launch_tc(const ssd_fwd_params &p, const Plan &plan, const Dims &d, 
     if (ins.main) cudaEventRecord(ins.main, stream);
     const int split = direct_split(p, s);
     if (split < 0) {
-        e = launch_walk_any<false>(p.dstate, s.KH, s.max_items, mX, mB, mC, mY, prm, stream);
+        e = launch_out(gnp, p.dstate, s.KH, s.max_items, mX, mB, mC, mY, prm, stream);
     } else {
         prm.n_items = split;
-        e = launch_walk_any<false>(p.dstate, 2, split, mX, mB, mC, mY, prm, stream);
+        e = launch_out(gnp, p.dstate, 2, split, mX, mB, mC, mY, prm, stream);
         if (e == cudaSuccess) {
             TcParams tail = prm;
             tail.direct_base = split * 2;
             tail.n_items = (s.max_items - split) * 2;
-            e = launch_walk_any<false>(p.dstate, 1, tail.n_items, mX, mB, mC, mY, tail, stream);
+            e = launch_out(gnp, p.dstate, 1, tail.n_items, mX, mB, mC, mY, tail, stream);
         }
     }
     if (ins.end) cudaEventRecord(ins.end, stream);

@@ -13,6 +13,10 @@ struct TcArgs {
     float *final_states;
     void *scratch;
     size_t scratch_bytes;
+    // gated norm of the block output (z == nullptr: plain y)
+    const void *z = nullptr;
+    const float *gn_w = nullptr, *gn_b = nullptr;
+    float gn_eps = 0.0f;
 };
 
 bool tc_supported(const ssd_fwd_params &p);
