@@ -152,6 +152,9 @@ constexpr size_t tc_smem_bytes()
 {
     return sizeof(TcSmem<NST>) + 1024;   // + alignment slack
 }
+// opt-in shared memory per block on sm_100 (227 KB)
+static_assert(tc_smem_bytes<64>() <= 232448 && tc_smem_bytes<128>() <= 232448 && tc_smem_bytes<256>() <= 232448,
+              "walk kernel shared memory exceeds the per-block limit");
 
 __device__ __forceinline__ void record_timeout(int *status) { set_status(status, kDevTimeout); }
 
@@ -496,7 +499,17 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             // L2 prefetch runs kPF blocks ahead of the shared-memory ring
             constexpr int kPF = STATE_ONLY ? 1 : (NST >= 256 ? 2 : kPrefetch);
             auto prefetch = [&](int c) {
-                const int row = it.tok0 + (STATE_ONLY ? nblk - 1 - c : c) * kQ;   // state-only: backwards
+                const int blk = STATE_ONLY ? nblk - 1 - c : c;
+                const int row = it.tok0 + blk * kQ;   // state-only: backwards
+                {
+                    // the block's dt rows (every head), read by the cumsum warp with plain loads:
+                    // 16-byte aligned and inside the segment
+                    const int rows = min(kQ, it.len - blk * kQ);
+                    const uintptr_t b0 = reinterpret_cast<uintptr_t>(prm.dt + (size_t)row * prm.H);
+                    const uintptr_t e0 = reinterpret_cast<uintptr_t>(prm.dt + (size_t)(row + rows) * prm.H);
+                    const uintptr_t a0 = (b0 + 15) & ~(uintptr_t)15, a1 = e0 & ~(uintptr_t)15;
+                    if (a1 > a0) prefetch_l2_bulk(reinterpret_cast<const void *>(a0), (uint32_t)(a1 - a0));
+                }
                 for (int b = 0; b < NST / 64; ++b) {
                     if (!STATE_ONLY) tma_prefetch_l2_2d(&mapC, g * NST + 64 * b, row);
                     tma_prefetch_l2_2d(&mapB, g * NST + 64 * b, row);

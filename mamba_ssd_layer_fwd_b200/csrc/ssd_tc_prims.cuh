@@ -134,6 +134,14 @@ __device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *map, int c
                  : "memory");
 }
 
+// Bring a contiguous byte range into L2 (no shared memory, no completion);
+// address and size multiples of 16.
+__device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+                 : "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
