@@ -486,9 +486,10 @@ def run_ours(args):
             del sfw
             torch.cuda.empty_cache()
 
-    backward = None
+    backward = decode = None
     if world == 1 and not args.no_sub_workloads:
         backward = measure_backward(ssd, args, dev, flush)
+        decode = measure_decode(ssd, args, dev, flush)
 
     if rank == 0:
         cpu = None
@@ -515,6 +516,7 @@ def run_ours(args):
             "wall_s_timed_region": wall,
             "workloads": subs,
             "backward": backward,
+            "decode": decode,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -591,6 +593,43 @@ def measure_backward(ssd, args, dev, flush, steps=10):
             "alg_bytes": nb, "frac_hbm": nb / (med * 1e-3) / 1e9 / peak, "path": "simt (CUDA cores, fp32)",
             "check": {"sequence": 0, "max_rel_err": errs, "tol": 1e-3,
                       "ok": bool(max(errs.values()) <= 1e-3)}}
+
+
+def measure_decode(ssd, args, dev, flush, steps=50):
+    """One ssd_decode_step over every row of decode_2p7b (64 rows of the 2.7B
+    layer shape, state resident), L2 flushed before each timed step; the
+    first step's y and state checked against the oracle's recurrence."""
+    import torch
+    import oracle
+    inp = ssd_inputs.make_inputs(ssd_inputs.workload("decode_2p7b"), seed=args.seed)
+    d = {k: torch.from_numpy(np.ascontiguousarray(inp[k][:, 0])).to(dev, torch.bfloat16) for k in ("x", "dt", "B", "C")}
+    A_log = torch.from_numpy(inp["A_log"]).to(dev)
+    D = torch.from_numpy(inp["D"]).to(dev)
+    state0 = torch.from_numpy(inp["initial_states"]).to(dev)
+    state = state0.clone()
+    y = torch.empty_like(d["x"])
+    stream = torch.cuda.current_stream()
+    ssd.ssd_decode_step(d["x"], d["dt"], A_log, d["B"], d["C"], D, state, y=y, stream=stream)
+    torch.cuda.synchronize()
+    y_ref, fin_ref = oracle.recurrence(inp)
+    ey = float(np.abs(y.double().cpu().numpy() - y_ref[:, 0]).max() / np.abs(y_ref).max())
+    ef = float(np.abs(state.double().cpu().numpy() - fin_ref).max() / np.abs(fin_ref).max())
+    ms = []
+    for _ in range(steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        ssd.ssd_decode_step(d["x"], d["dt"], A_log, d["B"], d["C"], D, state, y=y, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    med = statistics.median(ms)
+    nb = decode_bytes(inp)
+    peak, _ = measured_peaks()
+    rows = inp["x"].shape[0]
+    return {"workload": "decode_2p7b", "ms": _stats(ms), "tokens_per_s": rows / (med * 1e-3), "alg_bytes": nb,
+            "frac_hbm": nb / (med * 1e-3) / 1e9 / peak,
+            "check": {"max_rel_err_y": ey, "max_rel_err_state": ef, "tol": 2e-2, "ok": bool(ey <= 2e-2 and ef <= 2e-2)}}
 
 
 def fw_launches(ssd, inp, path):

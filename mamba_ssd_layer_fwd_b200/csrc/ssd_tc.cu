@@ -222,6 +222,9 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
     }
     // only non-final segments need end states (every sequence's, for a summary)
     if (STATE_ONLY && !prm.summary && it.seg >= it.nseg - 1) return;
+    // a launch queued behind this one as a programmatic dependent (the one-head items left
+    // after whole waves, which read nothing this launch writes) may start as SMs free up
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q = warp & 3;                             // SM sub-partition = TMEM lane quarter
@@ -1181,6 +1184,9 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
         tc_fence_after();
         tmem_dealloc(tb, 512);
     }
+    // launched as a programmatic dependent: do not finish before the launch ahead of this one,
+    // so that work queued after this launch sees both complete (immediate otherwise)
+    if (tid == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // ---------------------------------------------------------------- planning
@@ -1444,41 +1450,57 @@ TcPlanShape plan_shape(const ssd_fwd_params &p)
 template <int NST, int KH, bool SO, bool GN>
 cudaError_t launch_walk(int grid, const CUtensorMap &mX, const CUtensorMap &mB, const CUtensorMap &mC,
                         const CUtensorMap &mY,
-                        const TcParams &prm, cudaStream_t st, const GnParams &gnp = GnParams{})
+                        const TcParams &prm, cudaStream_t st, const GnParams &gnp = GnParams{}, bool overlap = false)
 {
     const size_t smem = tc_smem_bytes<NST>();
     cudaError_t e = cudaFuncSetAttribute(ssd_tc_walk<NST, KH, SO, GN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    ssd_tc_walk<NST, KH, SO, GN><<<grid, kThreadsTc, smem, st>>>(mX, mB, mC, mY, prm, gnp);
-    return cudaGetLastError();
+    if (!overlap) {
+        ssd_tc_walk<NST, KH, SO, GN><<<grid, kThreadsTc, smem, st>>>(mX, mB, mC, mY, prm, gnp);
+        return cudaGetLastError();
+    }
+    // programmatic dependent launch: may begin before the previous kernel on the stream has
+    // finished; only for work that reads nothing that kernel writes
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreadsTc);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, ssd_tc_walk<NST, KH, SO, GN>, mX, mB, mC, mY, prm, gnp);
 }
 
 template <int NST, bool SO, bool GN>
 cudaError_t launch_walk_kh(int KH, int grid, const CUtensorMap &mX, const CUtensorMap &mB, const CUtensorMap &mC,
                            const CUtensorMap &mY,
-                           const TcParams &prm, cudaStream_t st, const GnParams &gnp = GnParams{})
+                           const TcParams &prm, cudaStream_t st, const GnParams &gnp = GnParams{}, bool overlap = false)
 {
-    return KH == 2 ? launch_walk<NST, 2, SO, GN>(grid, mX, mB, mC, mY, prm, st, gnp)
-                   : launch_walk<NST, 1, SO, GN>(grid, mX, mB, mC, mY, prm, st, gnp);
+    return KH == 2 ? launch_walk<NST, 2, SO, GN>(grid, mX, mB, mC, mY, prm, st, gnp, overlap)
+                   : launch_walk<NST, 1, SO, GN>(grid, mX, mB, mC, mY, prm, st, gnp, overlap);
 }
 
 template <bool SO, bool GN = false>
 cudaError_t launch_walk_any(int N, int KH, int grid, const CUtensorMap &mX, const CUtensorMap &mB,
                             const CUtensorMap &mC, const CUtensorMap &mY, const TcParams &prm, cudaStream_t st,
-                            const GnParams &gnp = GnParams{})
+                            const GnParams &gnp = GnParams{}, bool overlap = false)
 {
-    if (N == 256) return launch_walk_kh<256, SO, GN>(KH, grid, mX, mB, mC, mY, prm, st, gnp);
-    return N == 128 ? launch_walk_kh<128, SO, GN>(KH, grid, mX, mB, mC, mY, prm, st, gnp)
-                    : launch_walk_kh<64, SO, GN>(KH, grid, mX, mB, mC, mY, prm, st, gnp);
+    if (N == 256) return launch_walk_kh<256, SO, GN>(KH, grid, mX, mB, mC, mY, prm, st, gnp, overlap);
+    return N == 128 ? launch_walk_kh<128, SO, GN>(KH, grid, mX, mB, mC, mY, prm, st, gnp, overlap)
+                    : launch_walk_kh<64, SO, GN>(KH, grid, mX, mB, mC, mY, prm, st, gnp, overlap);
 }
 
 // the output pass, with or without the gated norm epilogue
 cudaError_t launch_out(const GnParams &gnp, int N, int KH, int grid, const CUtensorMap &mX, const CUtensorMap &mB,
-                       const CUtensorMap &mC, const CUtensorMap &mY, const TcParams &prm, cudaStream_t st)
+                       const CUtensorMap &mC, const CUtensorMap &mY, const TcParams &prm, cudaStream_t st,
+                       bool overlap = false)
 {
-    return gnp.z ? launch_walk_any<false, true>(N, KH, grid, mX, mB, mC, mY, prm, st, gnp)
-                 : launch_walk_any<false, false>(N, KH, grid, mX, mB, mC, mY, prm, st);
+    return gnp.z ? launch_walk_any<false, true>(N, KH, grid, mX, mB, mC, mY, prm, st, gnp, overlap)
+                 : launch_walk_any<false, false>(N, KH, grid, mX, mB, mC, mY, prm, st, GnParams{}, overlap);
 }
 
 size_t align256(size_t v) { return (v + 255) / 256 * 256; }
@@ -1616,7 +1638,7 @@ cudaError_t launch_tc(const ssd_fwd_params &p, const Plan &plan, const Dims &d, 
             TcParams tail = prm;
             tail.direct_base = split * 2;
             tail.n_items = (s.max_items - split) * 2;
-            e = launch_out(gnp, p.dstate, 1, tail.n_items, mX, mB, mC, mY, tail, stream);
+            e = launch_out(gnp, p.dstate, 1, tail.n_items, mX, mB, mC, mY, tail, stream, /*overlap=*/true);
         }
     }
     if (ins.end) cudaEventRecord(ins.end, stream);
