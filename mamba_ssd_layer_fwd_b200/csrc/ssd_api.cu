@@ -71,7 +71,7 @@ Layout layout_of(const ssd_fwd_params &p, int path)
 {
     Layout L{};
     size_t off = 0;
-    L.status = off; off += kAlign;
+    L.status = off; off += kStatusRegion;
     L.count = off; off += kAlign;
     const size_t mc = (size_t)max_chunks_of(p);
     const size_t ns = (size_t)nseq_of(p);

@@ -34,6 +34,12 @@ struct SeqDesc {
     int len;
 };
 
+// The forward's workspace starts with this many bytes: the status word, and
+// from kSyncOffsetInts on, counters that CTAs of one launch use to wait for one
+// another (zeroed with the status word before such a launch).
+constexpr size_t kStatusRegion = 2048;
+constexpr int kSyncOffsetInts = 64;
+
 struct Plan {
     int *status;        // device status word
     int *count;         // number of valid chunk entries

@@ -48,6 +48,9 @@
 // passing between pieces of a sequence).
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+#include <atomic>
+
 #include "ssd_tc.cuh"
 #include "ssd_tc_prims.cuh"
 
@@ -122,6 +125,14 @@ __device__ __forceinline__ float softplus_fast(float v)
 }
 
 // --------------------------------------------------------------- smem layout
+// The mbarriers of one walk.
+struct TcBars {
+    uint64_t bc_full[2], bc_empty[2], x_full[2], x_empty[2], cs_full[kCsd], cs_empty[kCsd];
+    uint64_t cb_full, cb_empty, pm_full[2], pm_empty[2], hb_full, hb_empty, xw_full[2], xw_empty[2], xw_free[2];
+    uint64_t yo_full;
+    uint64_t h_ready[2], hs_full[2], y_full, yo_empty, yd_empty, drain_o, drain_s;
+};
+
 template <int NST>
 struct __align__(1024) TcSmem {
     static constexpr int kBoxes = NST / 64;
@@ -139,10 +150,7 @@ struct __align__(1024) TcSmem {
     int exact[kCsd];                   // 1: some 16-token chunk decays too fast for the factorised mask
     float alpha[kCsd];                 // exp(cs_last)
     float ldec[kCsd];                  // cs_last (natural log of the block decay)
-    uint64_t bc_full[2], bc_empty[2], x_full[2], x_empty[2], cs_full[kCsd], cs_empty[kCsd];
-    uint64_t cb_full, cb_empty, pm_full[2], pm_empty[2], hb_full, hb_empty, xw_full[2], xw_empty[2], xw_free[2];
-    uint64_t yo_full;
-    uint64_t h_ready[2], hs_full[2], y_full, yo_empty, yd_empty, drain_o, drain_s;
+    TcBars bar[2];                     // one barrier set per walk of the CTA
     uint32_t tmem_base;
     int abort;
 };
@@ -189,42 +197,19 @@ __device__ long long *g_trace = nullptr;
     } while (0)
 #endif
 
-template <int NST, int KH, bool STATE_ONLY, bool GN = false>
-__global__ void __launch_bounds__(kThreadsTc, 1)
-ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapB,
-            const __grid_constant__ CUtensorMap mapC, const __grid_constant__ CUtensorMap mapY, const TcParams prm,
-            const GnParams gnp)
+// One walk over a work item's segment: the state-only walk (end state from
+// zero, backwards) or the full walk (outputs and the end state), by the CTA's
+// 512 threads with barrier set Bb (initialised here), TMEM columns from tb.
+// srow: row of segstate / seglogdec that holds head it.h0 of this segment
+// (the heads of the item are srow .. srow + KH - 1).
+template <int NST, int KH, bool STATE_ONLY, bool GN>
+__device__ __forceinline__ void walk_body(const CUtensorMap &mapX, const CUtensorMap &mapB, const CUtensorMap &mapC,
+                                          const CUtensorMap &mapY, const TcParams &prm, const GnParams &gnp,
+                                          TcSmem<NST> &S, TcBars &Bb, const uint32_t tb, const TcItem &it,
+                                          const int item_idx, const int srow)
 {
-    extern __shared__ uint8_t smem_raw[];
-    // 1024-byte alignment (128-byte swizzle atoms) computed as an offset from the
-    // shared array itself, so every access below stays a shared-memory access
-    const uint32_t smem_pad = ((smem_u32(smem_raw) + 1023u) & ~1023u) - smem_u32(smem_raw);
-    TcSmem<NST> &S = *reinterpret_cast<TcSmem<NST> *>(smem_raw + smem_pad);
     // dstate 256 keeps more live registers: there the out-of-line wait call spills
     constexpr bool kInlW = NST >= 256;
-    const int item_idx = blockIdx.x;
-    TcItem it;
-    if (prm.items) {
-        if (item_idx >= *prm.count) return;
-        it = prm.items[item_idx];
-    } else {
-        if (item_idx >= prm.n_items) return;
-        const int g0 = prm.direct_base + item_idx * KH;
-        const int row = g0 / prm.H;
-        it.seq = row;
-        it.tok0 = row * prm.seqlen;
-        it.len = prm.seqlen;
-        it.gseg = row;
-        it.seg = 0;
-        it.nseg = 1;
-        it.h0 = g0 - row * prm.H;
-        it.pad = 0;
-    }
-    // only non-final segments need end states (every sequence's, for a summary)
-    if (STATE_ONLY && !prm.summary && it.seg >= it.nseg - 1) return;
-    // a launch queued behind this one as a programmatic dependent (the one-head items left
-    // after whole waves, which read nothing this launch writes) may start as SMs free up
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q = warp & 3;                             // SM sub-partition = TMEM lane quarter
@@ -270,42 +255,35 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
 
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&S.bc_full[i], 1);
-            mbar_init(&S.bc_empty[i], STATE_ONLY ? 1 : 2);    // state issuer (+ output issuer)
-            mbar_init(&S.x_full[i], 1);
-            mbar_init(&S.x_empty[i], STATE_ONLY ? 2 : 3);     // w o X warps (+ output issuer)
-            mbar_init(&S.xw_full[i], 2);
-            mbar_init(&S.xw_empty[i], kTmaY ? 4 : 1);       // epilogue warps, else the state issuer
-            mbar_init(&S.xw_free[i], 1);
-            mbar_init(&S.pm_full[i], kMaskWarps);
-            mbar_init(&S.pm_empty[i], 1);
-            mbar_init(&S.h_ready[i], 1);
-            mbar_init(&S.hs_full[i], 4);      // per head: H rescaled for its next block
+            mbar_init(&Bb.bc_full[i], 1);
+            mbar_init(&Bb.bc_empty[i], STATE_ONLY ? 1 : 2);    // state issuer (+ output issuer)
+            mbar_init(&Bb.x_full[i], 1);
+            mbar_init(&Bb.x_empty[i], STATE_ONLY ? 2 : 3);     // w o X warps (+ output issuer)
+            mbar_init(&Bb.xw_full[i], 2);
+            mbar_init(&Bb.xw_empty[i], kTmaY ? 4 : 1);       // epilogue warps, else the state issuer
+            mbar_init(&Bb.xw_free[i], 1);
+            mbar_init(&Bb.pm_full[i], kMaskWarps);
+            mbar_init(&Bb.pm_empty[i], 1);
+            mbar_init(&Bb.h_ready[i], 1);
+            mbar_init(&Bb.hs_full[i], 4);      // per head: H rescaled for its next block
         }
         for (int i = 0; i < kCsd; ++i) {
-            mbar_init(&S.cs_full[i], 32);
-            mbar_init(&S.cs_empty[i], STATE_ONLY ? 6 : 6 + kMaskWarps);
+            mbar_init(&Bb.cs_full[i], 32);
+            mbar_init(&Bb.cs_empty[i], STATE_ONLY ? 6 : 6 + kMaskWarps);
         }
-        mbar_init(&S.cb_full, 1);
-        mbar_init(&S.cb_empty, kMaskWarps);
-        mbar_init(&S.hb_full, 4);
-        mbar_init(&S.hb_empty, 1);
-        mbar_init(&S.y_full, 1);
-        mbar_init(&S.yo_full, 1);
-        mbar_init(&S.yo_empty, 4);
-        mbar_init(&S.yd_empty, 4);
-        mbar_init(&S.drain_o, 1);
-        mbar_init(&S.drain_s, 1);
-        S.abort = 0;
+        mbar_init(&Bb.cb_full, 1);
+        mbar_init(&Bb.cb_empty, kMaskWarps);
+        mbar_init(&Bb.hb_full, 4);
+        mbar_init(&Bb.hb_empty, 1);
+        mbar_init(&Bb.y_full, 1);
+        mbar_init(&Bb.yo_full, 1);
+        mbar_init(&Bb.yo_empty, 4);
+        mbar_init(&Bb.yd_empty, 4);
+        mbar_init(&Bb.drain_o, 1);
+        mbar_init(&Bb.drain_s, 1);
         mbar_fence_init();
     }
-    if (warp == 3) {
-        tmem_alloc(&S.tmem_base, 512);
-        tmem_relinquish();
-    }
     __syncthreads();
-    tc_fence_after();
-    const uint32_t tb = S.tmem_base;
 #ifdef SSD_TRACE
     const long long t_start = clock64();
     long long *const trace_buf = (blockIdx.x < kTraceCtas && !STATE_ONLY) ? g_trace : nullptr;
@@ -339,7 +317,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
 #pragma unroll
             for (int jj = 1; jj < KH; ++jj)
                 if (j == jj) A = Areg[jj];
-            if (u >= kCsd) ok = mbar_wait<kInlW>(&S.cs_empty[slot], ((u / kCsd) + 1) & 1, abort);
+            if (u >= kCsd) ok = mbar_wait<kInlW>(&Bb.cs_empty[slot], ((u / kCsd) + 1) & 1, abort);
             if (!ok) break;
             // lane owns tokens 4*lane .. 4*lane+3
             float dl[4], pre[4];
@@ -396,7 +374,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                 S.ldec[slot] = last;
                 S.exact[slot] = exact;
             }
-            mbar_arrive(&S.cs_full[slot]);
+            mbar_arrive(&Bb.cs_full[slot]);
             if (lane == 0) SSD_TRACE_EV(6, u);
         }
     } else if (warp == 1) {
@@ -412,13 +390,13 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             bool ok = true;
             for (int c = 0; c < nblk && ok; ++c) {
                 const int bs = c % kBR;
-                ok = mbar_wait<kInlW>(&S.bc_full[kSplitBC ? 1 : bs], (c / kBR) & 1, abort);
+                ok = mbar_wait<kInlW>(&Bb.bc_full[kSplitBC ? 1 : bs], (c / kBR) & 1, abort);
                 if (!ok) break;
                 const uint32_t sB = smem_u32(b_tile(bs));
                 if (kMergeSt) {
                     // both heads: w o X tiles 0 and 1 (u = 2c, 2c + 1) form one N = 128 operand
-                    ok = mbar_wait<kInlW>(&S.xw_full[0], c & 1, abort) && mbar_wait<kInlW>(&S.xw_full[1], c & 1, abort) &&
-                         (c > 0 || (mbar_wait<kInlW>(&S.hs_full[0], 0, abort) && mbar_wait<kInlW>(&S.hs_full[1], 0, abort)));
+                    ok = mbar_wait<kInlW>(&Bb.xw_full[0], c & 1, abort) && mbar_wait<kInlW>(&Bb.xw_full[1], c & 1, abort) &&
+                         (c > 0 || (mbar_wait<kInlW>(&Bb.hs_full[0], 0, abort) && mbar_wait<kInlW>(&Bb.hs_full[1], 0, abort)));
                     if (!ok) break;
                     tc_fence_after();
                     const uint64_t b0 = sdesc_sw128(smem_u32(xw_tile(0)), 16384, 1024);
@@ -432,20 +410,20 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                                         id_h2, 1);
                     }
                     if (leader) {
-                        umma_commit(&S.xw_empty[0]);
-                        umma_commit(&S.xw_empty[1]);
-                        umma_commit(&S.h_ready[0]);
-                        umma_commit(&S.h_ready[1]);
-                        umma_commit(&S.bc_empty[bs]);
+                        umma_commit(&Bb.xw_empty[0]);
+                        umma_commit(&Bb.xw_empty[1]);
+                        umma_commit(&Bb.h_ready[0]);
+                        umma_commit(&Bb.h_ready[1]);
+                        umma_commit(&Bb.bc_empty[bs]);
                     }
                     continue;
                 }
                 for (int j = 0; j < KH && ok; ++j) {
                     const int u = c * KH + j, wi = u % kXwR;
                     // state-only mode never rescales: hs_full[j] completes once, when the zeroed state is in place
-                    ok = mbar_wait<kInlW>(&S.xw_full[wi], (u / kXwR) & 1, abort) &&
-                         (STATE_ONLY ? (c > 0 || mbar_wait<kInlW>(&S.hs_full[j], 0, abort))
-                                     : mbar_wait<kInlW>(&S.hs_full[j], c & 1, abort));
+                    ok = mbar_wait<kInlW>(&Bb.xw_full[wi], (u / kXwR) & 1, abort) &&
+                         (STATE_ONLY ? (c > 0 || mbar_wait<kInlW>(&Bb.hs_full[j], 0, abort))
+                                     : mbar_wait<kInlW>(&Bb.hs_full[j], c & 1, abort));
                     SSD_TRACE_EV(15, u);
                     if (!ok) break;
                     tc_fence_after();
@@ -459,16 +437,16 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                                 umma_ss(tb + kColH + 64 * (j + KH * mt), desc_adv(a0, kk * 2048),
                                         desc_adv(b0, kk * 2048), id_h, 1);
                     }
-                    if (leader) umma_commit(kTmaY ? &S.xw_free[wi] : &S.xw_empty[wi]);
-                    if (leader) umma_commit(&S.h_ready[j]);
-                    if (kSplitBC && j == KH - 1 && leader) umma_commit(&S.bc_empty[1]);   // B of block c done
+                    if (leader) umma_commit(kTmaY ? &Bb.xw_free[wi] : &Bb.xw_empty[wi]);
+                    if (leader) umma_commit(&Bb.h_ready[j]);
+                    if (kSplitBC && j == KH - 1 && leader) umma_commit(&Bb.bc_empty[1]);   // B of block c done
                     SSD_TRACE_EV(4, u);
                     if (kYoOnState) {
                         // the accumulator is free once the epilogue has read the previous unit's
                         // Yo (its own columns) or Yd (columns shared with Yo)
-                        ok = mbar_wait<kInlW>(&S.hb_full, u & 1, abort) &&
-                             (u == 0 || mbar_wait<kInlW>(kSharedY ? &S.yd_empty : &S.yo_empty, (u - 1) & 1, abort)) &&
-                             (!kSplitBC || j > 0 || mbar_wait<kInlW>(&S.bc_full[0], c & 1, abort));
+                        ok = mbar_wait<kInlW>(&Bb.hb_full, u & 1, abort) &&
+                             (u == 0 || mbar_wait<kInlW>(kSharedY ? &Bb.yd_empty : &Bb.yo_empty, (u - 1) & 1, abort)) &&
+                             (!kSplitBC || j > 0 || mbar_wait<kInlW>(&Bb.bc_full[0], c & 1, abort));
                         if (!ok) break;
                         tc_fence_after();
                         const uint64_t c0 = sdesc_sw128(smem_u32(S.bc[bs][0][0]), 16, 1024);
@@ -479,15 +457,15 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                             if (leader)
                                 umma_ss(tb + kColYo, desc_adv(c0, off), desc_adv(h0, kk * 2048), id_y, kk > 0);
                         }
-                        if (leader) umma_commit(&S.hb_empty);
-                        if (leader) umma_commit(&S.yo_full);
+                        if (leader) umma_commit(&Bb.hb_empty);
+                        if (leader) umma_commit(&Bb.yo_full);
                         SSD_TRACE_EV(27, u);
                     }
                 }
-                if (leader) umma_commit(&S.bc_empty[kSplitBC ? 0 : bs]);   // (C of block c done)
+                if (leader) umma_commit(&Bb.bc_empty[kSplitBC ? 0 : bs]);   // (C of block c done)
             }
-            if (leader) umma_commit(&S.drain_s);
-            mbar_wait<kInlW>(&S.drain_s, 0, abort, 200000000ull);
+            if (leader) umma_commit(&Bb.drain_s);
+            mbar_wait<kInlW>(&Bb.drain_s, 0, abort, 200000000ull);
         }
     } else if (warp == 2) {
         // ------------------------------------------------------ TMA producer
@@ -522,10 +500,10 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             // split B/C stage: one half (1 = B, 0 = C) of block c
             auto load_half = [&](int c, int half) -> bool {
                 const int row = it.tok0 + (STATE_ONLY ? nblk - 1 - c : c) * kQ;   // state-only: backwards
-                if (c >= 1 && !mbar_wait<kInlW>(&S.bc_empty[half], (c + 1) & 1, abort)) return false;
-                mbar_arrive_expect_tx(&S.bc_full[half], (NST / 64) * 16384u);
+                if (c >= 1 && !mbar_wait<kInlW>(&Bb.bc_empty[half], (c + 1) & 1, abort)) return false;
+                mbar_arrive_expect_tx(&Bb.bc_full[half], (NST / 64) * 16384u);
                 for (int b = 0; b < NST / 64; ++b)
-                    tma_load_2d(S.bc[0][half][b], half ? &mapB : &mapC, &S.bc_full[half], g * NST + 64 * b, row);
+                    tma_load_2d(S.bc[0][half][b], half ? &mapB : &mapC, &Bb.bc_full[half], g * NST + 64 * b, row);
                 issued_bc[half] = c;
                 if (half == 0) SSD_TRACE_EV(0, c);
                 return true;
@@ -533,12 +511,12 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             auto load_bc = [&](int c) -> bool {
                 const int row = it.tok0 + (STATE_ONLY ? nblk - 1 - c : c) * kQ;   // state-only: backwards
                 const int bs = c % kBR;
-                if (c >= kBR && !mbar_wait<kInlW>(&S.bc_empty[bs], ((c / kBR) + 1) & 1, abort)) return false;
-                mbar_arrive_expect_tx(&S.bc_full[bs], kBcBytes);
+                if (c >= kBR && !mbar_wait<kInlW>(&Bb.bc_empty[bs], ((c / kBR) + 1) & 1, abort)) return false;
+                mbar_arrive_expect_tx(&Bb.bc_full[bs], kBcBytes);
                 uint8_t *bdst = b_tile(bs);
                 for (int b = 0; b < NST / 64; ++b) {
-                    if (!STATE_ONLY) tma_load_2d(S.bc[bs][0][b], &mapC, &S.bc_full[bs], g * NST + 64 * b, row);
-                    tma_load_2d(bdst + 16384 * b, &mapB, &S.bc_full[bs], g * NST + 64 * b, row);
+                    if (!STATE_ONLY) tma_load_2d(S.bc[bs][0][b], &mapC, &Bb.bc_full[bs], g * NST + 64 * b, row);
+                    tma_load_2d(bdst + 16384 * b, &mapB, &Bb.bc_full[bs], g * NST + 64 * b, row);
                 }
                 issued_bc[bs] = c;
                 SSD_TRACE_EV(0, c);
@@ -548,10 +526,10 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                 const int row = it.tok0 + (STATE_ONLY ? nblk - 1 - c : c) * kQ;   // state-only: backwards
                 for (int j = j0; j < j1; ++j) {
                     const int u = c * KH + j, xs = u & 1;
-                    if (u >= 2 && !mbar_wait<kInlW>(&S.x_empty[xs], ((u >> 1) + 1) & 1, abort)) return false;
+                    if (u >= 2 && !mbar_wait<kInlW>(&Bb.x_empty[xs], ((u >> 1) + 1) & 1, abort)) return false;
                     if (prm.withhold_x0 && item_idx == 0 && u == 0) continue;
-                    mbar_arrive_expect_tx(&S.x_full[xs], kBoxBytes);
-                    tma_load_2d(S.x[xs], &mapX, &S.x_full[xs], (it.h0 + j) * kP, row);
+                    mbar_arrive_expect_tx(&Bb.x_full[xs], kBoxBytes);
+                    tma_load_2d(S.x[xs], &mapX, &Bb.x_full[xs], (it.h0 + j) * kP, row);
                     issued_x[xs] = u;
                     SSD_TRACE_EV(1, u);
                 }
@@ -574,10 +552,10 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                 // drain: wait (bounded) for copies still in flight before the CTA exits
                 for (int i = 0; i < 2; ++i) {
                     if (kSplitBC && issued_bc[i] >= 0)
-                        mbar_wait<kInlW>(&S.bc_full[i], issued_bc[i] & 1, abort, 200000000ull);
+                        mbar_wait<kInlW>(&Bb.bc_full[i], issued_bc[i] & 1, abort, 200000000ull);
                     else if (i < kBR && issued_bc[i] >= 0)
-                        mbar_wait<kInlW>(&S.bc_full[i], (issued_bc[i] / kBR) & 1, abort, 200000000ull);
-                    if (issued_x[i] >= 0) mbar_wait<kInlW>(&S.x_full[i], (issued_x[i] >> 1) & 1, abort, 200000000ull);
+                        mbar_wait<kInlW>(&Bb.bc_full[i], (issued_bc[i] / kBR) & 1, abort, 200000000ull);
+                    if (issued_x[i] >= 0) mbar_wait<kInlW>(&Bb.x_full[i], (issued_x[i] >> 1) & 1, abort, 200000000ull);
                 }
             }
         }
@@ -592,11 +570,11 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             // CB = C_c B_c^T into the single CB accumulator
             auto issue_cb = [&](int c) -> bool {
                 const int bs = c % kSt;
-                if (!mbar_wait<kInlW>(&S.bc_full[bs], (c / kSt) & 1, abort)) return false;
-                if (kSplitBC && !mbar_wait<kInlW>(&S.bc_full[1], c & 1, abort)) return false;
-                if (c >= 1 && !mbar_wait<kInlW>(&S.cb_empty, (c - 1) & 1, abort)) return false;
+                if (!mbar_wait<kInlW>(&Bb.bc_full[bs], (c / kSt) & 1, abort)) return false;
+                if (kSplitBC && !mbar_wait<kInlW>(&Bb.bc_full[1], c & 1, abort)) return false;
+                if (c >= 1 && !mbar_wait<kInlW>(&Bb.cb_empty, (c - 1) & 1, abort)) return false;
                 // the previous block's last Pm lives in the CB columns until its Pm X is done
-                if (kInPlace && c >= 1 && !mbar_wait<kInlW>(&S.pm_empty[1], (c - 1) & 1, abort)) return false;
+                if (kInPlace && c >= 1 && !mbar_wait<kInlW>(&Bb.pm_empty[1], (c - 1) & 1, abort)) return false;
                 tc_fence_after();
                 const uint64_t a0 = sdesc_sw128(smem_u32(S.bc[bs][0][0]), 16, 1024);
                 const uint64_t b0 = sdesc_sw128(smem_u32(S.bc[bs][1][0]), 16, 1024);
@@ -605,11 +583,11 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                     const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
                     if (leader) umma_ss(tb + kColCB, desc_adv(a0, off), desc_adv(b0, off), id_cb, kk > 0);
                 }
-                if (leader) umma_commit(&S.cb_full);
+                if (leader) umma_commit(&Bb.cb_full);
                 if (kYoOnState && leader) {
                     // CB is this issuer's only use of B and C
-                    umma_commit(&S.bc_empty[0]);
-                    if (kSplitBC) umma_commit(&S.bc_empty[1]);
+                    umma_commit(&Bb.bc_empty[0]);
+                    if (kSplitBC) umma_commit(&Bb.bc_empty[1]);
                 }
                 SSD_TRACE_EV(2, c);
                 return true;
@@ -631,9 +609,9 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                     const int pph = kInPlace ? (c & 1) : ((u / kPmB) & 1);
                     // Yo = C Hbf^T (issued by the state issuer when kYoOnState)
                     if (!kYoOnState) {
-                        ok = mbar_wait<kInlW>(&S.hb_full, u & 1, abort);
+                        ok = mbar_wait<kInlW>(&Bb.hb_full, u & 1, abort);
                         SSD_TRACE_EV(14, u);
-                        ok = ok && (u == 0 || mbar_wait<kInlW>(&S.yo_empty, (u - 1) & 1, abort));
+                        ok = ok && (u == 0 || mbar_wait<kInlW>(&Bb.yo_empty, (u - 1) & 1, abort));
                         SSD_TRACE_EV(17, u);
                         if (!ok) break;
                         tc_fence_after();
@@ -643,7 +621,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                             const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
                             if (leader) umma_ss(tb + kColYo, desc_adv(a0, off), desc_adv(b0, kk * 2048), id_y, kk > 0);
                         }
-                        if (leader) umma_commit(&S.hb_empty);
+                        if (leader) umma_commit(&Bb.hb_empty);
                         SSD_TRACE_EV(3, u);
                     }
                     // the next block's CB runs while the mask warps finish this block's last head
@@ -653,10 +631,10 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                     }
                     // Yd = Pm X, once the accumulator is free: the previous Yd read, or (shared
                     // with Yo) this unit's Yo read
-                    ok = mbar_wait<kInlW>(&S.pm_full[pi], pph, abort) &&
-                         mbar_wait<kInlW>(&S.x_full[xs], (u >> 1) & 1, abort) &&
-                         (kSharedY ? mbar_wait<kInlW>(&S.yo_empty, u & 1, abort)
-                                   : (u == 0 || mbar_wait<kInlW>(&S.yd_empty, (u - 1) & 1, abort)));
+                    ok = mbar_wait<kInlW>(&Bb.pm_full[pi], pph, abort) &&
+                         mbar_wait<kInlW>(&Bb.x_full[xs], (u >> 1) & 1, abort) &&
+                         (kSharedY ? mbar_wait<kInlW>(&Bb.yo_empty, u & 1, abort)
+                                   : (u == 0 || mbar_wait<kInlW>(&Bb.yd_empty, (u - 1) & 1, abort)));
                     SSD_TRACE_EV(16, u);
                     if (!ok) break;
                     tc_fence_after();
@@ -668,16 +646,16 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                         const uint32_t acol = pm + kk * 8 + (ip && kk >= 4 ? 32u : 0u);
                         if (leader) umma_ts(tb + kColYd, acol, desc_adv(x0, kk * 2048), id_y, kk > 0);
                     }
-                    if (leader) umma_commit(&S.pm_empty[pi]);
-                    if (leader) umma_commit(&S.y_full);
-                    if (leader) umma_commit(&S.x_empty[xs]);
+                    if (leader) umma_commit(&Bb.pm_empty[pi]);
+                    if (leader) umma_commit(&Bb.y_full);
+                    if (leader) umma_commit(&Bb.x_empty[xs]);
                     SSD_TRACE_EV(5, u);
                 }
-                if (!kYoOnState && leader) umma_commit(&S.bc_empty[bs]);
+                if (!kYoOnState && leader) umma_commit(&Bb.bc_empty[bs]);
             }
             // every UMMA issued so far has completed before TMEM is released
-            if (leader) umma_commit(&S.drain_o);
-            mbar_wait<kInlW>(&S.drain_o, 0, abort, 200000000ull);
+            if (leader) umma_commit(&Bb.drain_o);
+            mbar_wait<kInlW>(&Bb.drain_o, 0, abort, 200000000ull);
         }
     } else if ((warp >= 4 && warp < 8) || warp == 10 || warp == 11) {
         // ------------------------------------------------------------- mask
@@ -696,18 +674,18 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             for (int j = 0; j < KH; ++j) Dreg[j] = prm.D ? prm.D[it.h0 + j] : 0.0f;
             bool ok = true;
             for (int c = 0; c < nblk && ok; ++c) {
-                ok = mbar_wait<kInlW>(&S.cb_full, c & 1, abort);
+                ok = mbar_wait<kInlW>(&Bb.cb_full, c & 1, abort);
                 if (!ok) break;
                 tc_fence_after();
                 for (int j = 0; j < KH; ++j) {
                     const int u = c * KH + j, slot = u % kCsd;
                     const bool ip = kInPlace && j == 1;    // written over the CB columns just read
                     const int pi = kInPlace ? j : u % kPmB;
-                    ok = mbar_wait<kInlW>(&S.cs_full[slot], (u / kCsd) & 1, abort);
+                    ok = mbar_wait<kInlW>(&Bb.cs_full[slot], (u / kCsd) & 1, abort);
                     if (kInPlace)
-                        ok = ok && (ip || c == 0 || mbar_wait<kInlW>(&S.pm_empty[0], (c - 1) & 1, abort));
+                        ok = ok && (ip || c == 0 || mbar_wait<kInlW>(&Bb.pm_empty[0], (c - 1) & 1, abort));
                     else
-                        ok = ok && (u < kPmB || mbar_wait<kInlW>(&S.pm_empty[pi], ((u / kPmB) + 1) & 1, abort));
+                        ok = ok && (u < kPmB || mbar_wait<kInlW>(&Bb.pm_empty[pi], ((u / kPmB) + 1) & 1, abort));
                     if (!ok) break;
                     tc_fence_after();
                     if (warp == 4 && lane == 0) SSD_TRACE_EV(7, u);
@@ -743,7 +721,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                             if (j == KH - 1 && pair == npairs - 1) {
                                 tc_fence_before();
                                 __syncwarp();
-                                if (lane == 0) mbar_arrive(&S.cb_empty);
+                                if (lane == 0) mbar_arrive(&Bb.cb_empty);
                             }
                             float m[32];
                             if (!exact) {
@@ -795,7 +773,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                     if (j == KH - 1 && npairs == 0) {           // rows with no work still release CB
                         tc_fence_before();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(&S.cb_empty);
+                        if (lane == 0) mbar_arrive(&Bb.cb_empty);
                     }
                     if (ip && q < 2) {
                         // rows 0..63: K steps 4-7 (columns 64-95 in place) lie above the diagonal; nothing
@@ -810,8 +788,8 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) {
-                        mbar_arrive(&S.pm_full[pi]);
-                        mbar_arrive(&S.cs_empty[slot]);
+                        mbar_arrive(&Bb.pm_full[pi]);
+                        mbar_arrive(&Bb.cs_empty[slot]);
                         if (warp == 4) SSD_TRACE_EV(8, u);
                     }
                 }
@@ -835,9 +813,9 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
         const int r0 = (warp - 8) * 64 + lane;          // rows r0 and r0 + 32
         for (int u = 0; u < nunits && ok; ++u) {
             const int slot = u % kCsd, xs = u & 1, wi = u % kXwR;
-            ok = mbar_wait<kInlW>(&S.cs_full[slot], (u / kCsd) & 1, abort) &&
-                 mbar_wait<kInlW>(&S.x_full[xs], (u >> 1) & 1, abort) &&
-                 (u < kXwR || mbar_wait<kInlW>(&S.xw_empty[wi], ((u / kXwR) + 1) & 1, abort));
+            ok = mbar_wait<kInlW>(&Bb.cs_full[slot], (u / kCsd) & 1, abort) &&
+                 mbar_wait<kInlW>(&Bb.x_full[xs], (u >> 1) & 1, abort) &&
+                 (u < kXwR || mbar_wait<kInlW>(&Bb.xw_empty[wi], ((u / kXwR) + 1) & 1, abort));
             if (!ok) break;
             if (warp == 8 && lane == 0) SSD_TRACE_EV(25, u);
             {
@@ -853,7 +831,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                     for (int ch = 0; ch < 8; ++ch)
                         v[rr][ch] = *reinterpret_cast<const uint4 *>(S.x[xs] + (r0 + 32 * rr) * 128 + ((ch * 16) ^ rot));
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&S.x_empty[xs]);   // X no longer read by this warp
+                if (lane == 0) mbar_arrive(&Bb.x_empty[xs]);   // X no longer read by this warp
 #pragma unroll
                 for (int rr = 0; rr < 2; ++rr) {
                     const int t = r0 + 32 * rr;
@@ -870,8 +848,8 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             fence_async_smem();
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(&S.xw_full[wi]);
-                mbar_arrive(&S.cs_empty[slot]);
+                mbar_arrive(&Bb.xw_full[wi]);
+                mbar_arrive(&Bb.cs_empty[slot]);
                 if (warp == 8) SSD_TRACE_EV(11, u);
             }
         }
@@ -880,14 +858,16 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
         const int t = q * 32 + lane;                   // TMEM lane: state row n / output row l
         const int N = NST;
         const size_t PN = (size_t)kP * N;
-        // initial state of every head: from the caller, from the segment scan, or zero
+        // initial state of every head: from the caller, from the segment scan, or zero.  Plain
+        // loads: a segment state written by another CTA of this launch (the segmented walk) was
+        // only ever read here through L2 (.cg) loads, so no stale line of it sits in L1
         for (int j = 0; j < KH; ++j) {
             const int h = it.h0 + j;
             // state-only mode measures each segment from a zero state
             const float *src = nullptr;
             if (!STATE_ONLY) {
                 if (it.nseg > 1)
-                    src = prm.segstate + ((size_t)it.gseg * prm.H + h) * PN;
+                    src = prm.segstate + (size_t)(srow + j) * PN;
                 else if (prm.init)
                     src = prm.init + ((size_t)it.seq * prm.H + h) * PN;
             }
@@ -914,8 +894,8 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
         auto epilogue = [&](int v) -> bool {
             const int c = v / KH, j = v % KH, slot = v % kCsd;
             // Yd and Yo in one accumulator: Yo is read first, then Pm X may write Yd
-            if (!kSharedY && !mbar_wait<kInlW>(&S.y_full, v & 1, abort)) return false;
-            if (kYoOnState && !mbar_wait<kInlW>(&S.yo_full, v & 1, abort)) return false;
+            if (!kSharedY && !mbar_wait<kInlW>(&Bb.y_full, v & 1, abort)) return false;
+            if (kYoOnState && !mbar_wait<kInlW>(&Bb.yo_full, v & 1, abort)) return false;
             tc_fence_after();
             if (warp == 12 && lane == 0) SSD_TRACE_EV(12, v);
             const int valid = min(kQ, it.len - c * kQ);
@@ -929,10 +909,10 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&S.yo_empty);
+            if (lane == 0) mbar_arrive(&Bb.yo_empty);
             if (warp == 12 && lane == 0) SSD_TRACE_EV(26, v);
             if (kSharedY) {
-                if (!mbar_wait<kInlW>(&S.y_full, v & 1, abort)) return false;
+                if (!mbar_wait<kInlW>(&Bb.y_full, v & 1, abort)) return false;
                 tc_fence_after();
                 if (warp == 12 && lane == 0) SSD_TRACE_EV(17, v);
             }
@@ -941,7 +921,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             uint8_t *stage = S.xw[wi] + q * 32 * 128;     // this warp's 32 rows, 128-byte swizzled
             const bool via_tma = kTmaY && valid == kQ;
             // the slot's w o X tile is free once the state UMMA of unit v has completed
-            if (kTmaY && !mbar_wait<kInlW>(&S.xw_free[wi], (v / kXwD) & 1, abort)) return false;
+            if (kTmaY && !mbar_wait<kInlW>(&Bb.xw_free[wi], (v / kXwD) & 1, abort)) return false;
             if (GN) {
                 // Mamba-2 block output (Sec. 7.1): g = y * silu(z), staged as bf16 while the
                 // statistics accumulate (shifted by the row's first g), then normalised over the
@@ -958,7 +938,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                     if (h0 == kP - 32) {
                         tc_fence_before();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(&S.yd_empty);
+                        if (lane == 0) mbar_arrive(&Bb.yd_empty);
                     }
                     if (row_ok) {
 #pragma unroll
@@ -1025,7 +1005,7 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                 if (h0 == kP - 32) {
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&S.yd_empty);
+                    if (lane == 0) mbar_arrive(&Bb.yd_empty);
                 }
                 if (via_tma || t < valid) {
 #pragma unroll
@@ -1058,8 +1038,8 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                     bulk_wait_read_all();
                 }
                 if (warp == 12) SSD_TRACE_EV(24, v);
-                if (kTmaY) mbar_arrive(&S.xw_empty[wi]);
-                mbar_arrive(&S.cs_empty[slot]);
+                if (kTmaY) mbar_arrive(&Bb.xw_empty[wi]);
+                mbar_arrive(&Bb.cs_empty[slot]);
             }
             if (warp == 12 && lane == 0) SSD_TRACE_EV(13, v);
             return true;
@@ -1076,22 +1056,22 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                 if (c == 0) {
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&S.hs_full[j]);   // the zeroed state is in place
+                    if (lane == 0) mbar_arrive(&Bb.hs_full[j]);   // the zeroed state is in place
                 }
-                ok = mbar_wait<kInlW>(&S.cs_full[slot], (u / kCsd) & 1, abort);
+                ok = mbar_wait<kInlW>(&Bb.cs_full[slot], (u / kCsd) & 1, abort);
                 if (!ok) break;
                 const float ld = S.ldec[slot];
 #pragma unroll
                 for (int jj = 0; jj < KH; ++jj)
                     if (j == jj) ldec_sum[jj] += ld;
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&S.cs_empty[slot]);
+                if (lane == 0) mbar_arrive(&Bb.cs_empty[slot]);
                 continue;
             }
-            ok = mbar_wait<kInlW>(&S.cs_full[slot], (u / kCsd) & 1, abort) &&
-                 (c == 0 || mbar_wait<kInlW>(&S.h_ready[j], (c - 1) & 1, abort));
+            ok = mbar_wait<kInlW>(&Bb.cs_full[slot], (u / kCsd) & 1, abort) &&
+                 (c == 0 || mbar_wait<kInlW>(&Bb.h_ready[j], (c - 1) & 1, abort));
             if (!ok) break;
-            if (!STATE_ONLY) ok = (u == 0 || mbar_wait<kInlW>(&S.hb_empty, (u - 1) & 1, abort));
+            if (!STATE_ONLY) ok = (u == 0 || mbar_wait<kInlW>(&Bb.hb_empty, (u - 1) & 1, abort));
             if (!ok) break;
             tc_fence_after();
             if (warp == 12 && lane == 0) SSD_TRACE_EV(9, u);
@@ -1136,9 +1116,9 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-                if (!STATE_ONLY) mbar_arrive(&S.hb_full);
-                mbar_arrive(&S.hs_full[j]);
-                if (STATE_ONLY) mbar_arrive(&S.cs_empty[slot]);
+                if (!STATE_ONLY) mbar_arrive(&Bb.hb_full);
+                mbar_arrive(&Bb.hs_full[j]);
+                if (STATE_ONLY) mbar_arrive(&Bb.cs_empty[slot]);
             }
             if (warp == 12 && lane == 0) SSD_TRACE_EV(10, u);
             if (!STATE_ONLY && u >= 1) ok = epilogue(u - 1);
@@ -1146,13 +1126,13 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
         // end of the segment: the state after the last token
         if (ok) {
             for (int j = 0; j < KH; ++j) {
-                ok = mbar_wait<kInlW>(&S.h_ready[j], (nblk - 1) & 1, abort);
+                ok = mbar_wait<kInlW>(&Bb.h_ready[j], (nblk - 1) & 1, abort);
                 if (!ok) break;
                 tc_fence_after();
                 const int h = it.h0 + j;
                 float *dst = nullptr;
                 if (STATE_ONLY)
-                    dst = prm.segstate + ((size_t)(prm.summary ? it.seq : it.gseg) * prm.H + h) * PN;
+                    dst = prm.segstate + (size_t)(srow + j) * PN;
                 else if (it.seg == it.nseg - 1 && prm.final_states)
                     dst = prm.final_states + ((size_t)it.seq * prm.H + h) * PN;
 #pragma unroll
@@ -1171,21 +1151,222 @@ ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CU
                     }
                 }
                 if (STATE_ONLY && t == 0)
-                    prm.seglogdec[(size_t)(prm.summary ? it.seq : it.gseg) * prm.H + h] = ldec_sum[j];
+                    prm.seglogdec[srow + j] = ldec_sum[j];
             }
         }
         if (kTmaY && lane == 0) bulk_wait_all();       // this warp's y stores have landed
     }
 
-    // ------------------------------------------------------------ teardown
+}
+
+// Shared-memory carve-out and the 512-column TMEM allocation of a walk CTA;
+// every kernel below starts with it and ends with walk_teardown.
+template <int NST>
+__device__ __forceinline__ TcSmem<NST> &walk_smem()
+{
+    extern __shared__ uint8_t smem_raw[];
+    // 1024-byte alignment (128-byte swizzle atoms) computed as an offset from the
+    // shared array itself, so every access below stays a shared-memory access
+    const uint32_t smem_pad = ((smem_u32(smem_raw) + 1023u) & ~1023u) - smem_u32(smem_raw);
+    return *reinterpret_cast<TcSmem<NST> *>(smem_raw + smem_pad);
+}
+
+template <int NST>
+__device__ __forceinline__ uint32_t walk_setup(TcSmem<NST> &S)
+{
+    if (threadIdx.x == 0) S.abort = 0;
+    if (threadIdx.x / 32 == 3) {
+        tmem_alloc(&S.tmem_base, 512);
+        tmem_relinquish();
+    }
     __syncthreads();
-    if (S.abort && tid == 0) record_timeout(prm.status);
-    if (warp == 3) {
+    tc_fence_after();
+    return S.tmem_base;
+}
+
+template <int NST>
+__device__ __forceinline__ void walk_teardown(TcSmem<NST> &S, uint32_t tb, int *status)
+{
+    __syncthreads();
+    if (S.abort && threadIdx.x == 0) record_timeout(status);
+    if (threadIdx.x / 32 == 3) {
         tc_fence_after();
         tmem_dealloc(tb, 512);
     }
+}
+
+template <int NST, int KH, bool STATE_ONLY, bool GN = false>
+__global__ void __launch_bounds__(kThreadsTc, 1)
+ssd_tc_walk(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapB,
+            const __grid_constant__ CUtensorMap mapC, const __grid_constant__ CUtensorMap mapY,
+            const __grid_constant__ TcParams prm, const __grid_constant__ GnParams gnp)
+{
+    TcSmem<NST> &S = walk_smem<NST>();
+    const int item_idx = blockIdx.x;
+    TcItem it;
+    if (prm.items) {
+        if (item_idx >= *prm.count) return;
+        it = prm.items[item_idx];
+    } else {
+        if (item_idx >= prm.n_items) return;
+        const int g0 = prm.direct_base + item_idx * KH;
+        const int row = g0 / prm.H;
+        it.seq = row;
+        it.tok0 = row * prm.seqlen;
+        it.len = prm.seqlen;
+        it.gseg = row;
+        it.seg = 0;
+        it.nseg = 1;
+        it.h0 = g0 - row * prm.H;
+        it.pad = 0;
+    }
+    // only non-final segments need end states (every sequence's, for a summary)
+    if (STATE_ONLY && !prm.summary && it.seg >= it.nseg - 1) return;
+    // a launch queued behind this one as a programmatic dependent (the one-head items left
+    // after whole waves, which read nothing this launch writes) may start as SMs free up
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const uint32_t tb = walk_setup(S);
+    const int srow = (prm.summary ? it.seq : it.gseg) * prm.H + it.h0;
+    walk_body<NST, KH, STATE_ONLY, GN>(mapX, mapB, mapC, mapY, prm, gnp, S, S.bar[0], tb, it, item_idx, srow);
+    walk_teardown(S, tb, prm.status);
     // launched as a programmatic dependent: do not finish before the launch ahead of this one,
     // so that work queued after this launch sees both complete (immediate otherwise)
+    if (threadIdx.x == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Wait (bounded, 2 s) until the counter at p reaches target; acquire ordering.
+__device__ __noinline__ bool counter_wait(const int *p, int target, volatile int *abort)
+{
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        int v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+        if (v >= target) return true;
+        if ((it & 63u) == 0) {
+            if (*abort) return false;
+            if (globaltimer_ns() - t0 > 2000000000ull) {
+                *abort = 1;
+                return false;
+            }
+        }
+        __nanosleep(100);
+    }
+}
+
+// Segments of equal-length rows in one launch (Sec. 8.2, state passing
+// between pieces of a sequence).  CTA (pair, seg) of a (row, head block) pair
+// cut into fp.nseg segments: (1) a non-final segment measures its end state
+// from zero (the state-only walk) and publishes it; (2) once every non-final
+// segment of the pair has published, the pair's nseg CTAs each chain one slice
+// of the states through the segments, replacing segment k's state by the state
+// entering segment k (the caller's initial state for k = 0); (3) once every
+// slice is chained, every CTA runs the full walk of its segment from its
+// entering state.  The waits between CTAs need every CTA of the pair resident
+// at once: the grid is at most one CTA per SM, launched cooperatively, and
+// every wait is bounded.
+struct FuseParams {
+    int *ctr;        // [pairs][2] arrival counters, zero before the launch
+    int pair_base;   // flattened (row, head block) index of the launch's first pair
+    int nseg;        // segments per pair (>= 2)
+    int seg_len;     // tokens of every segment but the last (the last takes the rest)
+};
+
+template <int NST, int KH, bool GN = false>
+__global__ void __launch_bounds__(kThreadsTc, 1)
+ssd_tc_fused(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapB,
+             const __grid_constant__ CUtensorMap mapC, const __grid_constant__ CUtensorMap mapY,
+             const __grid_constant__ TcParams prm, const __grid_constant__ GnParams gnp, const FuseParams fp)
+{
+    TcSmem<NST> &S = walk_smem<NST>();
+    const int tid = threadIdx.x;
+    const int pl = blockIdx.x / fp.nseg, seg = blockIdx.x - pl * fp.nseg;
+    const int n_hb = prm.H / KH;
+    const int pair = fp.pair_base + pl, row = pair / n_hb;
+    TcItem it;
+    it.seq = row;
+    it.tok0 = row * prm.seqlen + seg * fp.seg_len;
+    it.len = seg < fp.nseg - 1 ? fp.seg_len : prm.seqlen - (fp.nseg - 1) * fp.seg_len;
+    it.gseg = pl * fp.nseg + seg;
+    it.seg = seg;
+    it.nseg = fp.nseg;
+    it.h0 = (pair - row * n_hb) * KH;
+    it.pad = 0;
+    // segment states of the launch: [pair][segment][KH heads][P x N], decays [pair][segment][KH]
+    const int srow = it.gseg * KH;
+    const uint32_t tb = walk_setup(S);
+    if (seg < fp.nseg - 1)
+        walk_body<NST, KH, true, false>(mapX, mapB, mapC, mapY, prm, gnp, S, S.bar[0], tb, it, blockIdx.x, srow);
+    tc_fence_before();      // the first walk's tensor-memory accesses come before the second walk's
+    __syncthreads();
+
+    constexpr int PN = kP * NST;
+    int *const ctr = fp.ctr + 2 * pl;
+    if (tid == 0 && !S.abort) {
+        if (seg < fp.nseg - 1) {
+            __threadfence();
+            atomicAdd(ctr, 1);
+        }
+        counter_wait(ctr, fp.nseg - 1, &S.abort);
+        __threadfence();
+    }
+    __syncthreads();
+    if (!S.abort) {
+        // this CTA's slice of the pair's KH x P x N state elements, in whole 128-byte lines
+        // (float4 units), chained through the segments in place
+        constexpr int kTot4 = KH * PN / 4;
+        const int per4 = ((kTot4 + fp.nseg - 1) / fp.nseg + 7) / 8 * 8;
+        const int b4 = seg * per4, e4 = min(kTot4, b4 + per4);
+        const int srow0 = pl * fp.nseg * KH;
+        for (int i4 = b4 + tid; i4 < e4; i4 += kThreadsTc) {
+            const int e = i4 * 4, j = e / PN, idx = e - j * PN;
+            float4 hv = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            if (prm.init) {
+                // the caller's buffer: element loads (no alignment beyond 4 bytes assumed)
+                const float *ip = prm.init + ((size_t)row * prm.H + it.h0 + j) * PN + idx;
+                hv = make_float4(__ldcg(ip), __ldcg(ip + 1), __ldcg(ip + 2), __ldcg(ip + 3));
+            }
+            constexpr int kGroup = 8;
+            for (int k0 = 0; k0 < fp.nseg; k0 += kGroup) {
+                float4 sv[kGroup];
+                float dk[kGroup];
+#pragma unroll
+                for (int i = 0; i < kGroup; ++i) {
+                    const int k = k0 + i;
+                    const bool has = k < fp.nseg - 1;
+                    const int sr = srow0 + k * KH + j;
+                    sv[i] = has ? __ldcg(reinterpret_cast<const float4 *>(prm.segstate + (size_t)sr * PN + idx))
+                                : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                    dk[i] = has ? __expf(__ldcg(prm.seglogdec + sr)) : 0.0f;
+                }
+#pragma unroll
+                for (int i = 0; i < kGroup; ++i) {
+                    const int k = k0 + i;
+                    if (k < fp.nseg) {
+                        const int sr = srow0 + k * KH + j;
+                        __stcg(reinterpret_cast<float4 *>(prm.segstate + (size_t)sr * PN + idx), hv);
+                        hv.x = fmaf(dk[i], hv.x, sv[i].x);
+                        hv.y = fmaf(dk[i], hv.y, sv[i].y);
+                        hv.z = fmaf(dk[i], hv.z, sv[i].z);
+                        hv.w = fmaf(dk[i], hv.w, sv[i].w);
+                    }
+                }
+            }
+        }
+    }
+    __syncthreads();
+    if (tid == 0 && !S.abort) {
+        __threadfence();
+        atomicAdd(ctr + 1, 1);
+        counter_wait(ctr + 1, fp.nseg, &S.abort);
+        __threadfence();
+    }
+    __syncthreads();
+    tc_fence_after();
+    if (!S.abort)
+        walk_body<NST, KH, false, GN>(mapX, mapB, mapC, mapY, prm, gnp, S, S.bar[1], tb, it, blockIdx.x, srow);
+    walk_teardown(S, tb, prm.status);
+    // launched behind whole waves of the plain walk as a programmatic dependent: finish only
+    // after that launch, so that work queued after this one sees both complete
     if (tid == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
@@ -1503,7 +1684,136 @@ cudaError_t launch_out(const GnParams &gnp, int N, int KH, int grid, const CUten
                  : launch_walk_any<false, false>(N, KH, grid, mX, mB, mC, mY, prm, st, GnParams{}, overlap);
 }
 
+template <int NST, int KH, bool GN>
+cudaError_t launch_fused_t(int grid, const CUtensorMap &mX, const CUtensorMap &mB, const CUtensorMap &mC,
+                           const CUtensorMap &mY, const TcParams &prm, const GnParams &gnp, const FuseParams &fp,
+                           bool after_walk, cudaStream_t st)
+{
+    const size_t smem = tc_smem_bytes<NST>();
+    cudaError_t e = cudaFuncSetAttribute(ssd_tc_fused<NST, KH, GN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreadsTc);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    if (after_walk) {
+        // behind whole waves of the plain walk, which writes nothing this launch reads: start as
+        // SMs free up (the grid is at most one CTA per SM, so every CTA becomes resident)
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+    } else {
+        // the CTAs of a pair wait for one another: all resident at once
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, ssd_tc_fused<NST, KH, GN>, mX, mB, mC, mY, prm, gnp, fp);
+}
+
+template <int NST, bool GN>
+cudaError_t launch_fused_kh(int KH, int grid, const CUtensorMap &mX, const CUtensorMap &mB, const CUtensorMap &mC,
+                            const CUtensorMap &mY, const TcParams &prm, const GnParams &gnp, const FuseParams &fp,
+                            bool after_walk, cudaStream_t st)
+{
+    return KH == 2 ? launch_fused_t<NST, 2, GN>(grid, mX, mB, mC, mY, prm, gnp, fp, after_walk, st)
+                   : launch_fused_t<NST, 1, GN>(grid, mX, mB, mC, mY, prm, gnp, fp, after_walk, st);
+}
+
+template <bool GN>
+cudaError_t launch_fused_n(int N, int KH, int grid, const CUtensorMap &mX, const CUtensorMap &mB,
+                           const CUtensorMap &mC, const CUtensorMap &mY, const TcParams &prm, const GnParams &gnp,
+                           const FuseParams &fp, bool after_walk, cudaStream_t st)
+{
+    if (N == 256) return launch_fused_kh<256, GN>(KH, grid, mX, mB, mC, mY, prm, gnp, fp, after_walk, st);
+    return N == 128 ? launch_fused_kh<128, GN>(KH, grid, mX, mB, mC, mY, prm, gnp, fp, after_walk, st)
+                    : launch_fused_kh<64, GN>(KH, grid, mX, mB, mC, mY, prm, gnp, fp, after_walk, st);
+}
+
 size_t align256(size_t v) { return (v + 255) / 256 * 256; }
+
+// SMs of the current device, looked up once per device.
+int device_sms()
+{
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return kPlanSMs;
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = kPlanSMs;
+        cache[dev].store(n, std::memory_order_relaxed);
+    }
+    return n;
+}
+
+// Schedule of equal-length rows (no cu_seqlens): work item = (row, block of KH
+// heads), taken from the block index.  Whole waves of the SMs walk whole rows in
+// one launch; the pairs left over either join that launch (a last partial
+// wave), or run as one-head items in a second launch, or are cut into nseg
+// segments each and run by the single-launch segmented walk (ssd_tc_fused),
+// whichever a cost model in block steps of one SM prefers: a whole row costs
+// nblk, a one-head row about 0.6 nblk (started as SMs free up), a row cut into
+// segments of L blocks (the last one the rest) (1 + r) L + 6: every segment's
+// full walk starts after the slowest state-only walk (r: its cost per block
+// relative to the full walk; measured 0.4 at dstate 256, taken 0.5 below),
+// plus about 6 blocks for the second pipeline fill, the exchange and the drains
+// (measured on one B200: 6 to 8).
+struct UniformPlan {
+    int full;      // items of the whole-row launch (from item 0)
+    int tail1;     // one-head items of the second launch (the pairs after `full`), 0 = none
+    int pairs;     // pairs of the segmented launch (the pairs after `full`), 0 = none
+    int nseg, seg_len;
+};
+
+UniformPlan uniform_plan(const ssd_fwd_params &p, const TcPlanShape &s)
+{
+    UniformPlan u{};
+    const long long items = (long long)p.batch * s.n_hb;
+    const long long sms = std::min(kPlanSMs, device_sms());
+    const long long nblk = (p.seqlen + kQ - 1) / kQ;
+    const long long full = items / sms * sms, left = items - full;
+    u.full = (int)items;
+    if (left == 0 || nblk < 2) return u;
+    double best = (double)nblk;
+    int mode = 0;
+    if (s.KH == 2 && full > 0 && 0.6 * (double)nblk < best) {
+        best = 0.6 * (double)nblk;
+        mode = 1;
+    }
+    const double r = p.dstate >= 256 ? 0.4 : 0.5;
+    const long long nmax = std::min<long long>(std::min<long long>(sms / left, nblk), 64);
+    long long bn = 0, bl = 0;
+    for (long long n = 2; n <= nmax; ++n) {
+        const long long L = (nblk + n - 1) / n;
+        if (nblk - (n - 1) * L < 1) continue;     // the last segment would be empty
+        const double c = (1.0 + r) * (double)L + 6.0;
+        if (c < best - 1e-9) {
+            best = c;
+            mode = 2;
+            bn = n;
+            bl = L;
+        }
+    }
+    if (mode == 1) {
+        u.full = (int)full;
+        u.tail1 = (int)(2 * left);
+    } else if (mode == 2) {
+        u.full = (int)full;
+        u.pairs = (int)left;
+        u.nseg = (int)bn;
+        u.seg_len = (int)(bl * kQ);
+    }
+    return u;
+}
+
+size_t fused_state_bytes(const ssd_fwd_params &p, const TcPlanShape &s, const UniformPlan &u)
+{
+    const size_t rows = (size_t)u.pairs * u.nseg * s.KH;
+    return align256(rows * kP * p.dstate * sizeof(float)) + align256(rows * sizeof(float));
+}
 
 }  // namespace
 
@@ -1517,6 +1827,7 @@ bool tc_supported(const ssd_fwd_params &p)
 size_t tc_workspace_bytes(const ssd_fwd_params &p)
 {
     const TcPlanShape s = plan_shape(p);
+    if (p.num_seqs == 0) return fused_state_bytes(p, s, uniform_plan(p, s));
     size_t b = align256(sizeof(TcItem) * (size_t)s.max_items);
     if (s.segmented) {
         b += align256((size_t)s.max_segments * p.nheads * kP * p.dstate * sizeof(float));
@@ -1527,37 +1838,100 @@ size_t tc_workspace_bytes(const ssd_fwd_params &p)
     return b;
 }
 
-// Equal-length rows that need no segmentation: every work item is (row, head
-// block) and the walk derives it from its block index, so no planner runs.
-bool direct_items(const ssd_fwd_params &p, const TcPlanShape &s)
-{
-    return p.num_seqs == 0 && !s.segmented && (long long)p.batch * p.seqlen > 0;
-}
-
-// Direct items with two heads each that do not fill whole waves of the SMs:
-// the first whole waves run as two-head items, the pairs left over as twice as
-// many one-head items in a second launch, which take about half as long (a
-// last round of a few two-head items would leave most SMs idle for a whole
-// item).  Returns the number of two-head items of the first launch, or -1
-// for a single launch.
-int direct_split(const ssd_fwd_params &p, const TcPlanShape &s)
-{
-    if (!direct_items(p, s) || s.KH != 2) return -1;
-    const int waves = s.max_items / kPlanSMs;
-    if (waves < 1 || s.max_items % kPlanSMs == 0) return -1;
-    return waves * kPlanSMs;
-}
-
 int tc_launch_count(const ssd_fwd_params &p)
 {
     const TcPlanShape s = plan_shape(p);
-    return s.segmented ? 4 : direct_items(p, s) ? (direct_split(p, s) >= 0 ? 2 : 1) : 2;
+    if (p.num_seqs == 0) {
+        const UniformPlan u = uniform_plan(p, s);
+        return (u.full > 0 ? 1 : 0) + (u.tail1 > 0 || u.pairs > 0 ? 1 : 0);
+    }
+    return s.segmented ? 4 : 2;
 }
+
+namespace {
+// Equal-length rows: see uniform_plan.
+cudaError_t launch_tc_uniform(const ssd_fwd_params &p, const Plan &plan, const TcArgs &a, const TcPlanShape &s,
+                              TcParams prm, const GnParams &gnp, cudaStream_t stream, const Instr &ins)
+{
+    const UniformPlan u = uniform_plan(p, s);
+    const long long tokens = (long long)p.batch * p.seqlen;
+    // the status word, and the segmented launch's counters (one pair each)
+    cudaError_t e = cudaMemsetAsync(plan.status, 0, sizeof(int) * (kSyncOffsetInts + 2 * (size_t)u.pairs), stream);
+    if (e != cudaSuccess || tokens == 0) return e;
+    if (2 * (size_t)u.pairs > kStatusRegion / sizeof(int) - kSyncOffsetInts) return cudaErrorInvalidValue;
+    CUtensorMap mX, mB, mC, mY;
+    // y has x's layout; its map moves 32-row slabs (one per epilogue warp)
+    if (!make_map(&mX, a.x, (uint64_t)p.nheads * kP, (uint64_t)tokens) ||
+        !make_map(&mY, a.y, (uint64_t)p.nheads * kP, (uint64_t)tokens, 32) ||
+        !make_map(&mB, a.B, (uint64_t)p.ngroups * p.dstate, (uint64_t)tokens) ||
+        !make_map(&mC, a.C, (uint64_t)p.ngroups * p.dstate, (uint64_t)tokens))
+        return cudaErrorInvalidValue;
+    prm.items = nullptr;
+    prm.direct_base = 0;
+    if (u.pairs > 0) {
+        char *ws = static_cast<char *>(a.scratch);
+        const size_t rows = (size_t)u.pairs * u.nseg * s.KH;
+        prm.segstate = reinterpret_cast<float *>(ws);
+        prm.seglogdec = reinterpret_cast<float *>(ws + align256(rows * kP * p.dstate * sizeof(float)));
+    }
+    // one launch holds every phase of the work, so the output pass is the whole forward
+    if (ins.begin) cudaEventRecord(ins.begin, stream);
+    if (ins.main) cudaEventRecord(ins.main, stream);
+    if (u.full > 0) {
+        prm.n_items = u.full;
+        e = launch_out(gnp, p.dstate, s.KH, u.full, mX, mB, mC, mY, prm, stream);
+    }
+    if (e == cudaSuccess && u.tail1 > 0) {
+        TcParams tail = prm;
+        tail.direct_base = u.full * 2;
+        tail.n_items = u.tail1;
+        e = launch_out(gnp, p.dstate, 1, u.tail1, mX, mB, mC, mY, tail, stream, /*overlap=*/true);
+    }
+    if (e == cudaSuccess && u.pairs > 0) {
+        FuseParams fp;
+        fp.ctr = plan.status + kSyncOffsetInts;
+        fp.pair_base = u.full;
+        fp.nseg = u.nseg;
+        fp.seg_len = u.seg_len;
+        const int grid = u.pairs * u.nseg;
+        e = gnp.z ? launch_fused_n<true>(p.dstate, s.KH, grid, mX, mB, mC, mY, prm, gnp, fp, u.full > 0, stream)
+                  : launch_fused_n<false>(p.dstate, s.KH, grid, mX, mB, mC, mY, prm, gnp, fp, u.full > 0, stream);
+    }
+    if (ins.end) cudaEventRecord(ins.end, stream);
+    return e;
+}
+}  // namespace
 
 cudaError_t launch_tc(const ssd_fwd_params &p, const Plan &plan, const Dims &d, const TcArgs &a,
                       cudaStream_t stream, const Instr &ins)
 {
     const TcPlanShape s = plan_shape(p);
+    TcParams prm;
+    prm.dt = static_cast<const __nv_bfloat16 *>(a.dt);
+    prm.A_log = a.A_log;
+    prm.D = a.D;
+    prm.init = a.init;
+    prm.y = static_cast<__nv_bfloat16 *>(a.y);
+    prm.final_states = a.final_states;
+    prm.segstate = nullptr;
+    prm.seglogdec = nullptr;
+    prm.items = nullptr;
+    prm.count = plan.count;
+    prm.n_items = 0;
+    prm.direct_base = 0;
+    prm.seqlen = p.seqlen;
+    prm.status = plan.status;
+    prm.H = p.nheads;
+    prm.G = p.ngroups;
+    prm.N = p.dstate;
+    prm.heads_per_group = d.heads_per_group;
+    prm.dt_softplus = p.dt_softplus;
+    prm.withhold_x0 = ins.withhold_first_tile != 0;
+    prm.summary = 0;
+    GnParams gnp{static_cast<const __nv_bfloat16 *>(a.z), a.gn_w, a.gn_b, a.gn_eps};
+    if (p.num_seqs == 0) return launch_tc_uniform(p, plan, a, s, prm, gnp, stream, ins);
+
+    // packed sequences (cu_seqlens): the planner builds the work items on the device
     char *ws = static_cast<char *>(a.scratch);
     TcItem *items = reinterpret_cast<TcItem *>(ws);
     size_t off = align256(sizeof(TcItem) * (size_t)s.max_items);
@@ -1573,17 +1947,9 @@ cudaError_t launch_tc(const ssd_fwd_params &p, const Plan &plan, const Dims &d, 
     const long long tokens = (long long)p.batch * p.seqlen;
     const int PN = kP * p.dstate;
     const int nseq = plan.nseq;
-    const bool direct = direct_items(p, s);
-    cudaError_t e;
-    if (direct) {
-        // the status word is all the planner would have initialised
-        e = cudaMemsetAsync(plan.status, 0, sizeof(int), stream);
-    } else {
-        tc_plan_kernel<<<1, 1024, 0, stream>>>(a.cu_seqlens, nseq, p.seqlen, s.seg_len, s.n_hb, s.KH, items,
-                                               plan.count, s.max_items, plan.status, a.init, a.final_states,
-                                               p.nheads, PN, seqseg);
-        e = cudaGetLastError();
-    }
+    tc_plan_kernel<<<1, 1024, 0, stream>>>(a.cu_seqlens, nseq, p.seqlen, s.seg_len, s.n_hb, s.KH, items, plan.count,
+                                           s.max_items, plan.status, a.init, a.final_states, p.nheads, PN, seqseg);
+    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || tokens == 0) return e;
 
     CUtensorMap mX, mB, mC, mY;
@@ -1594,29 +1960,10 @@ cudaError_t launch_tc(const ssd_fwd_params &p, const Plan &plan, const Dims &d, 
         !make_map(&mC, a.C, (uint64_t)p.ngroups * p.dstate, (uint64_t)tokens))
         return cudaErrorInvalidValue;
 
-    TcParams prm;
-    prm.dt = static_cast<const __nv_bfloat16 *>(a.dt);
-    prm.A_log = a.A_log;
-    prm.D = a.D;
-    prm.init = a.init;
-    prm.y = static_cast<__nv_bfloat16 *>(a.y);
-    prm.final_states = a.final_states;
     prm.segstate = segstate;
     prm.seglogdec = seglogdec;
-    prm.items = direct ? nullptr : items;
-    prm.count = plan.count;
+    prm.items = items;
     prm.n_items = s.max_items;
-    prm.direct_base = 0;
-    prm.seqlen = p.seqlen;
-    prm.status = plan.status;
-    prm.H = p.nheads;
-    prm.G = p.ngroups;
-    prm.N = p.dstate;
-    prm.heads_per_group = d.heads_per_group;
-    prm.dt_softplus = p.dt_softplus;
-    prm.withhold_x0 = ins.withhold_first_tile != 0;
-    prm.summary = 0;
-    GnParams gnp{static_cast<const __nv_bfloat16 *>(a.z), a.gn_w, a.gn_b, a.gn_eps};
 
     if (ins.begin) cudaEventRecord(ins.begin, stream);
     if (s.segmented) {
@@ -1628,19 +1975,7 @@ cudaError_t launch_tc(const ssd_fwd_params &p, const Plan &plan, const Dims &d, 
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (ins.main) cudaEventRecord(ins.main, stream);
-    const int split = direct_split(p, s);
-    if (split < 0) {
-        e = launch_out(gnp, p.dstate, s.KH, s.max_items, mX, mB, mC, mY, prm, stream);
-    } else {
-        prm.n_items = split;
-        e = launch_out(gnp, p.dstate, 2, split, mX, mB, mC, mY, prm, stream);
-        if (e == cudaSuccess) {
-            TcParams tail = prm;
-            tail.direct_base = split * 2;
-            tail.n_items = (s.max_items - split) * 2;
-            e = launch_out(gnp, p.dstate, 1, tail.n_items, mX, mB, mC, mY, tail, stream, /*overlap=*/true);
-        }
-    }
+    e = launch_out(gnp, p.dstate, s.KH, s.max_items, mX, mB, mC, mY, prm, stream);
     if (ins.end) cudaEventRecord(ins.end, stream);
     return e;
 }

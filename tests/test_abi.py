@@ -129,8 +129,8 @@ def _tc_params(batch, seqlen, nheads, dstate, ngroups=1, num_seqs=0):
 def test_tensor_path_work_split(lib):
     """Host-side work planning of the tensor-core path (no GPU needed): how
     many kernels one forward launches for each kind of problem."""
-    # 8 x 80 heads: 320 two-head items = 2 whole waves of 148 + 24 pairs run as
-    # 48 one-head items in a second launch; no planner kernel
+    # 8 x 80 heads: 320 two-head items = 2 whole waves of 148 in one launch; the
+    # 24 pairs left over as 48 one-head items in a second launch
     p = _tc_params(8, 2048, 80, 128)
     assert ssd.resolved_path(p) == "tensor"
     assert ssd.launch_count(p) == 2
@@ -138,8 +138,11 @@ def test_tensor_path_work_split(lib):
     assert ssd.launch_count(_tc_params(148, 256, 2, 64)) == 1
     # one short row: one item, one launch
     assert ssd.launch_count(_tc_params(1, 128, 2, 64)) == 1
-    # a 16K-token row with 32 heads: cut into segments (planner, state pass, scan, walk)
-    assert ssd.launch_count(_tc_params(1, 16384, 32, 256, ngroups=8)) == 4
+    # a 16K-token row with 32 heads: 16 pairs cut into 9 segments, state-only walks,
+    # exchange and full walks in one launch
+    assert ssd.launch_count(_tc_params(1, 16384, 32, 256, ngroups=8)) == 1
+    # 160 two-head items of 3 blocks: 148 whole rows + 24 one-head items
+    assert ssd.launch_count(_tc_params(2, 300, 160, 64)) == 2
     # packed variable-length batch: planner + walk when there are enough items for
     # the SMs (16 x 24 here), + state pass + scan when it must be cut (one sequence)
     assert ssd.launch_count(_tc_params(1, 32768, 48, 128, num_seqs=16)) == 2

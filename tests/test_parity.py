@@ -135,6 +135,37 @@ def test_tail_items_split_into_single_heads():
     check_full(inp, path="tensor")
 
 
+def _plan(inp):
+    """(launches, workspace bytes) of the tensor path for these inputs."""
+    import mamba_ssd_layer_fwd_b200 as ssd
+    from _helpers import to_device
+    t = to_device(inp)
+    p = ssd.params_for(t["x"], t["B"], 256, None, True, "tensor")
+    return ssd.launch_count(p), ssd.workspace_size(p)
+
+
+@pytest.mark.parametrize("N,G,H,seqlen", [(128, 2, 4, 1000), (256, 1, 2, 1300), (64, 1, 6, 1500), (128, 1, 3, 1400)])
+def test_segmented_single_launch(N, G, H, seqlen):
+    """Equal-length rows with fewer (row, head block) pairs than SMs: every pair is
+    cut into segments (the last one ragged) and one launch runs the state-only
+    walks, the exchange of segment states and the full walks (Sec. 8.2); with
+    initial and final states, two-head and one-head items (H = 3)."""
+    inp = small_inputs(batch=2, seqlen=seqlen, H=H, P=64, N=N, G=G, Q=256, init=True, seed=N + H + seqlen)
+    launches, ws = _plan(inp)
+    assert launches == 1 and ws >= 2 * 64 * N * 4     # one launch, with segment states in the workspace
+    check_full(inp, path="tensor")
+
+
+def test_segmented_tail_after_whole_waves():
+    """152 two-head items of 32 blocks on 148 SMs: 148 walk whole rows, the 4
+    pairs left over are cut into segments and run by the single-launch segmented
+    walk, started as SMs free up behind the first launch."""
+    inp = small_inputs(batch=4, seqlen=4096, H=76, P=64, N=64, G=1, Q=256, init=True, seed=16)
+    launches, ws = _plan(inp)
+    assert launches == 2 and ws >= 2 * 64 * 64 * 4
+    check_full(inp, path="tensor")
+
+
 def test_zero_length_batch_passes_initial_state():
     inp = small_inputs(batch=2, seqlen=0, H=2, P=64, N=64, G=1, Q=256, init=True, seed=8)
     y, fin = run_gpu(inp)
@@ -214,6 +245,33 @@ def test_device_wait_timeout_reported():
     assert rc == 0
     assert lib.ssd_get_status(ws.data_ptr(), st) == -4      # SSD_ERR_TIMEOUT
     # the same context keeps working
+    check_full(inp, path="tensor")
+
+
+def test_segment_exchange_timeout_reported():
+    """The waits between CTAs of the single-launch segmented walk are bounded too:
+    work item 0 withholds a tile, so segment 0 never publishes its state; the
+    other segments' exchange waits run out (about 2 s), every CTA frees TMEM and
+    exits, and the host reads SSD_ERR_TIMEOUT; the context stays usable."""
+    import ctypes
+    import torch
+    import mamba_ssd_layer_fwd_b200 as ssd
+    from _helpers import to_device
+    inp = small_inputs(batch=1, seqlen=3000, H=2, P=64, N=256, G=1, Q=256, init=True, seed=13)
+    assert _plan(inp)[0] == 1
+    t = to_device(inp)
+    p = ssd.params_for(t["x"], t["B"], 256, None, True, "tensor")
+    ins = ssd.make_instrumentation(withhold_first_tile=True)
+    lib = ssd.library()
+    ws = torch.empty(ssd.workspace_size(p), dtype=torch.uint8, device="cuda")
+    y = torch.empty_like(t["x"])
+    st = torch.cuda.current_stream().cuda_stream or None
+    rc = lib.ssd_fwd_instrumented(ctypes.byref(p), t["x"].data_ptr(), t["dt"].data_ptr(), t["A_log"].data_ptr(),
+                                  t["B"].data_ptr(), t["C"].data_ptr(), t["D"].data_ptr(),
+                                  t["initial_states"].data_ptr(), None, y.data_ptr(), None, ws.data_ptr(),
+                                  ws.numel(), st, ctypes.byref(ins))
+    assert rc == 0
+    assert lib.ssd_get_status(ws.data_ptr(), st) == -4      # SSD_ERR_TIMEOUT
     check_full(inp, path="tensor")
 
 
