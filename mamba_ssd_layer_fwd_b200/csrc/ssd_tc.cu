@@ -50,6 +50,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <cstddef>
 
 #include "ssd_tc.cuh"
 #include "ssd_tc_prims.cuh"
@@ -131,6 +132,7 @@ struct TcBars {
     uint64_t cb_full, cb_empty, pm_full[2], pm_empty[2], hb_full, hb_empty, xw_full[2], xw_empty[2], xw_free[2];
     uint64_t yo_full;
     uint64_t h_ready[2], hs_full[2], y_full, yo_empty, yd_empty, drain_o, drain_s;
+    uint64_t xs_full[4], xs_empty[4], xws_full[4];   // state-only mode's X ring (w o X in place)
 };
 
 template <int NST>
@@ -247,8 +249,19 @@ __device__ __forceinline__ void walk_body(const CUtensorMap &mapX, const CUtenso
     // the heads' states are adjacent per 128-row tile (column kColH + 64 (j + KH mt)) and so are
     // their w o X tiles (at dstate 256 in the bf16(H) tile, which state-only mode does not use)
     constexpr bool kMergeSt = STATE_ONLY && KH == 2;
-    constexpr int kXwR = (STATE_ONLY && kXwD == 1) ? 2 : kXwD;     // w o X ring depth
-    auto xw_tile = [&](int i) -> uint8_t * { return (STATE_ONLY && kXwD == 1) ? S.hbf + 16384 * i : S.xw[i]; };
+    constexpr int kXwR = kXwD;                                      // w o X ring depth (full walk)
+    auto xw_tile = [&](int i) -> uint8_t * { return S.xw[i]; };
+    // X ring: two slots; in state-only mode four (barriers xs_*), laid over the x, w o X and
+    // (dstate 256) bf16(H) tiles, contiguous and otherwise unused there, with w o X written
+    // over X in place and the slot freed by the state UMMA, so X loads run two blocks ahead
+    constexpr int kXR = STATE_ONLY ? 4 : 2;
+    static_assert(offsetof(TcSmem<NST>, xw) == offsetof(TcSmem<NST>, x) + sizeof(S.x) &&
+                      offsetof(TcSmem<NST>, hbf) == offsetof(TcSmem<NST>, xw) + sizeof(S.xw) &&
+                      sizeof(S.x) + sizeof(S.xw) + sizeof(S.hbf) >= 4 * 16384,
+                  "the state-only X ring needs four contiguous 16 KB tiles");
+    auto x_tile = [&](int i) -> uint8_t * { return STATE_ONLY ? S.x[0] + 16384 * i : S.x[i]; };
+    uint64_t *const x_full_b = STATE_ONLY ? Bb.xs_full : Bb.x_full;
+    uint64_t *const x_empty_b = STATE_ONLY ? Bb.xs_empty : Bb.x_empty;
     auto b_tile = [&](int stage) -> uint8_t * {
         return (STATE_ONLY && kSt == 1) ? S.bc[0][stage][0] : S.bc[stage][1][0];
     };
@@ -281,6 +294,12 @@ __device__ __forceinline__ void walk_body(const CUtensorMap &mapX, const CUtenso
         mbar_init(&Bb.yd_empty, 4);
         mbar_init(&Bb.drain_o, 1);
         mbar_init(&Bb.drain_s, 1);
+        if (STATE_ONLY)
+            for (int i = 0; i < 4; ++i) {
+                mbar_init(&Bb.xs_full[i], 1);
+                mbar_init(&Bb.xs_empty[i], 1);     // the state UMMA
+                mbar_init(&Bb.xws_full[i], 2);     // w o X warps
+            }
         mbar_fence_init();
     }
     __syncthreads();
@@ -289,7 +308,10 @@ __device__ __forceinline__ void walk_body(const CUtensorMap &mapX, const CUtenso
     long long *const trace_buf = (blockIdx.x < kTraceCtas && !STATE_ONLY) ? g_trace : nullptr;
 #endif
 
-    if (warp == 0) {
+    // state-only mode with two heads: the idle mask warp 4 takes the second head's units, so the
+    // cumsum (about a global-load latency plus ~1k cycles per unit) keeps pace with the walk
+    constexpr bool kCs2 = STATE_ONLY && KH == 2;
+    if (warp == 0 || (kCs2 && warp == 4)) {
         // ----------------------------------------------------------- cumsum
         // dt of a unit is loaded before waiting for its ring slot.
         const int H = prm.H;
@@ -302,7 +324,7 @@ __device__ __forceinline__ void walk_body(const CUtensorMap &mapX, const CUtenso
 #pragma unroll
         for (int j = 0; j < KH; ++j) rsum[j] = 0.0f;
         bool ok = true;
-        for (int u = 0; u < nunits && ok; ++u) {
+        for (int u = kCs2 && warp == 4 ? 1 : 0; u < nunits && ok; u += kCs2 ? 2 : 1) {
             const int c = STATE_ONLY ? nblk - 1 - u / KH : u / KH, j = u % KH, slot = u % kCsd;
             const int row0 = it.tok0 + c * kQ;
             const int valid = min(kQ, it.len - c * kQ);
@@ -394,12 +416,13 @@ __device__ __forceinline__ void walk_body(const CUtensorMap &mapX, const CUtenso
                 if (!ok) break;
                 const uint32_t sB = smem_u32(b_tile(bs));
                 if (kMergeSt) {
-                    // both heads: w o X tiles 0 and 1 (u = 2c, 2c + 1) form one N = 128 operand
-                    ok = mbar_wait<kInlW>(&Bb.xw_full[0], c & 1, abort) && mbar_wait<kInlW>(&Bb.xw_full[1], c & 1, abort) &&
+                    // both heads: the w o X tiles of u = 2c, 2c + 1 (adjacent slots) form one N = 128 operand
+                    const int s0 = (2 * c) % kXR, ph = ((2 * c) / kXR) & 1;
+                    ok = mbar_wait<kInlW>(&Bb.xws_full[s0], ph, abort) && mbar_wait<kInlW>(&Bb.xws_full[s0 + 1], ph, abort) &&
                          (c > 0 || (mbar_wait<kInlW>(&Bb.hs_full[0], 0, abort) && mbar_wait<kInlW>(&Bb.hs_full[1], 0, abort)));
                     if (!ok) break;
                     tc_fence_after();
-                    const uint64_t b0 = sdesc_sw128(smem_u32(xw_tile(0)), 16384, 1024);
+                    const uint64_t b0 = sdesc_sw128(smem_u32(x_tile(s0)), 16384, 1024);
 #pragma unroll
                     for (int mt = 0; mt < kMT; ++mt) {
                         const uint64_t a0 = sdesc_sw128(sB + mt * 32768, lbo_m, 1024);
@@ -410,8 +433,8 @@ __device__ __forceinline__ void walk_body(const CUtensorMap &mapX, const CUtenso
                                         id_h2, 1);
                     }
                     if (leader) {
-                        umma_commit(&Bb.xw_empty[0]);
-                        umma_commit(&Bb.xw_empty[1]);
+                        umma_commit(&Bb.xs_empty[s0]);
+                        umma_commit(&Bb.xs_empty[s0 + 1]);
                         umma_commit(&Bb.h_ready[0]);
                         umma_commit(&Bb.h_ready[1]);
                         umma_commit(&Bb.bc_empty[bs]);
@@ -419,15 +442,18 @@ __device__ __forceinline__ void walk_body(const CUtensorMap &mapX, const CUtenso
                     continue;
                 }
                 for (int j = 0; j < KH && ok; ++j) {
-                    const int u = c * KH + j, wi = u % kXwR;
+                    const int u = c * KH + j;
+                    // w o X: its own ring, or (state-only mode) in place in the X ring
+                    const int wi = STATE_ONLY ? u % kXR : u % kXwR;
                     // state-only mode never rescales: hs_full[j] completes once, when the zeroed state is in place
-                    ok = mbar_wait<kInlW>(&Bb.xw_full[wi], (u / kXwR) & 1, abort) &&
+                    ok = (STATE_ONLY ? mbar_wait<kInlW>(&Bb.xws_full[wi], (u / kXR) & 1, abort)
+                                     : mbar_wait<kInlW>(&Bb.xw_full[wi], (u / kXwR) & 1, abort)) &&
                          (STATE_ONLY ? (c > 0 || mbar_wait<kInlW>(&Bb.hs_full[j], 0, abort))
                                      : mbar_wait<kInlW>(&Bb.hs_full[j], c & 1, abort));
                     SSD_TRACE_EV(15, u);
                     if (!ok) break;
                     tc_fence_after();
-                    const uint64_t b0 = sdesc_sw128(smem_u32(xw_tile(wi)), 16384, 1024);
+                    const uint64_t b0 = sdesc_sw128(smem_u32(STATE_ONLY ? x_tile(wi) : xw_tile(wi)), 16384, 1024);
 #pragma unroll
                     for (int mt = 0; mt < kMT; ++mt) {
                         const uint64_t a0 = sdesc_sw128(sB + mt * 32768, lbo_m, 1024);
@@ -437,7 +463,7 @@ __device__ __forceinline__ void walk_body(const CUtensorMap &mapX, const CUtenso
                                 umma_ss(tb + kColH + 64 * (j + KH * mt), desc_adv(a0, kk * 2048),
                                         desc_adv(b0, kk * 2048), id_h, 1);
                     }
-                    if (leader) umma_commit(kTmaY ? &Bb.xw_free[wi] : &Bb.xw_empty[wi]);
+                    if (leader) umma_commit(STATE_ONLY ? &Bb.xs_empty[wi] : kTmaY ? &Bb.xw_free[wi] : &Bb.xw_empty[wi]);
                     if (leader) umma_commit(&Bb.h_ready[j]);
                     if (kSplitBC && j == KH - 1 && leader) umma_commit(&Bb.bc_empty[1]);   // B of block c done
                     SSD_TRACE_EV(4, u);
@@ -475,7 +501,9 @@ __device__ __forceinline__ void walk_body(const CUtensorMap &mapX, const CUtenso
             if (!STATE_ONLY) tma_prefetch_desc(&mapC);
             constexpr uint32_t kBoxBytes = 16384;
             constexpr uint32_t kBcBytes = (STATE_ONLY ? 1 : 2) * (NST / 64) * kBoxBytes;
-            int issued_bc[2] = {-1, -1}, issued_x[2] = {-1, -1};
+            int issued_bc[2] = {-1, -1}, issued_x[kXR];
+#pragma unroll
+            for (int i = 0; i < kXR; ++i) issued_x[i] = -1;
             bool ok = true;
             // L2 prefetch runs kPF blocks ahead of the shared-memory ring
             constexpr int kPF = STATE_ONLY ? 1 : (NST >= 256 ? 2 : kPrefetch);
@@ -525,11 +553,11 @@ __device__ __forceinline__ void walk_body(const CUtensorMap &mapX, const CUtenso
             auto load_x = [&](int c, int j0, int j1) -> bool {
                 const int row = it.tok0 + (STATE_ONLY ? nblk - 1 - c : c) * kQ;   // state-only: backwards
                 for (int j = j0; j < j1; ++j) {
-                    const int u = c * KH + j, xs = u & 1;
-                    if (u >= 2 && !mbar_wait<kInlW>(&Bb.x_empty[xs], ((u >> 1) + 1) & 1, abort)) return false;
+                    const int u = c * KH + j, xs = u % kXR;
+                    if (u >= kXR && !mbar_wait<kInlW>(&x_empty_b[xs], ((u / kXR) + 1) & 1, abort)) return false;
                     if (prm.withhold_x0 && item_idx == 0 && u == 0) continue;
-                    mbar_arrive_expect_tx(&Bb.x_full[xs], kBoxBytes);
-                    tma_load_2d(S.x[xs], &mapX, &Bb.x_full[xs], (it.h0 + j) * kP, row);
+                    mbar_arrive_expect_tx(&x_full_b[xs], kBoxBytes);
+                    tma_load_2d(x_tile(xs), &mapX, &x_full_b[xs], (it.h0 + j) * kP, row);
                     issued_x[xs] = u;
                     SSD_TRACE_EV(1, u);
                 }
@@ -555,8 +583,9 @@ __device__ __forceinline__ void walk_body(const CUtensorMap &mapX, const CUtenso
                         mbar_wait<kInlW>(&Bb.bc_full[i], issued_bc[i] & 1, abort, 200000000ull);
                     else if (i < kBR && issued_bc[i] >= 0)
                         mbar_wait<kInlW>(&Bb.bc_full[i], (issued_bc[i] / kBR) & 1, abort, 200000000ull);
-                    if (issued_x[i] >= 0) mbar_wait<kInlW>(&Bb.x_full[i], (issued_x[i] >> 1) & 1, abort, 200000000ull);
                 }
+                for (int i = 0; i < kXR; ++i)
+                    if (issued_x[i] >= 0) mbar_wait<kInlW>(&x_full_b[i], (issued_x[i] / kXR) & 1, abort, 200000000ull);
             }
         }
     } else if (warp == 3) {
@@ -812,10 +841,10 @@ __device__ __forceinline__ void walk_body(const CUtensorMap &mapX, const CUtenso
         bool ok = true;
         const int r0 = (warp - 8) * 64 + lane;          // rows r0 and r0 + 32
         for (int u = 0; u < nunits && ok; ++u) {
-            const int slot = u % kCsd, xs = u & 1, wi = u % kXwR;
+            const int slot = u % kCsd, xs = u % kXR, wi = u % kXwR;
             ok = mbar_wait<kInlW>(&Bb.cs_full[slot], (u / kCsd) & 1, abort) &&
-                 mbar_wait<kInlW>(&Bb.x_full[xs], (u >> 1) & 1, abort) &&
-                 (u < kXwR || mbar_wait<kInlW>(&Bb.xw_empty[wi], ((u / kXwR) + 1) & 1, abort));
+                 mbar_wait<kInlW>(&x_full_b[xs], (u / kXR) & 1, abort) &&
+                 (STATE_ONLY || u < kXwR || mbar_wait<kInlW>(&Bb.xw_empty[wi], ((u / kXwR) + 1) & 1, abort));
             if (!ok) break;
             if (warp == 8 && lane == 0) SSD_TRACE_EV(25, u);
             {
@@ -829,9 +858,11 @@ __device__ __forceinline__ void walk_body(const CUtensorMap &mapX, const CUtenso
                 for (int rr = 0; rr < 2; ++rr)
 #pragma unroll
                     for (int ch = 0; ch < 8; ++ch)
-                        v[rr][ch] = *reinterpret_cast<const uint4 *>(S.x[xs] + (r0 + 32 * rr) * 128 + ((ch * 16) ^ rot));
+                        v[rr][ch] = *reinterpret_cast<const uint4 *>(x_tile(xs) + (r0 + 32 * rr) * 128 + ((ch * 16) ^ rot));
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&Bb.x_empty[xs]);   // X no longer read by this warp
+                if (!STATE_ONLY && lane == 0) mbar_arrive(&Bb.x_empty[xs]);   // X no longer read by this warp
+                // w o X: into its ring, or in place (this thread's own rows only)
+                uint8_t *const dst_tile = STATE_ONLY ? x_tile(xs) : xw_tile(wi);
 #pragma unroll
                 for (int rr = 0; rr < 2; ++rr) {
                     const int t = r0 + 32 * rr;
@@ -841,14 +872,14 @@ __device__ __forceinline__ void walk_body(const CUtensorMap &mapX, const CUtenso
                         __nv_bfloat162 *pv = reinterpret_cast<__nv_bfloat162 *>(&v[rr][ch]);
 #pragma unroll
                         for (int i = 0; i < 4; ++i) pv[i] = __hmul2(pv[i], ws2);
-                        *reinterpret_cast<uint4 *>(xw_tile(wi) + t * 128 + ((ch * 16) ^ rot)) = v[rr][ch];
+                        *reinterpret_cast<uint4 *>(dst_tile + t * 128 + ((ch * 16) ^ rot)) = v[rr][ch];
                     }
                 }
             }
             fence_async_smem();
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(&Bb.xw_full[wi]);
+                mbar_arrive(STATE_ONLY ? &Bb.xws_full[xs] : &Bb.xw_full[wi]);
                 mbar_arrive(&Bb.cs_empty[slot]);
                 if (warp == 8) SSD_TRACE_EV(11, u);
             }
@@ -1123,10 +1154,14 @@ __device__ __forceinline__ void walk_body(const CUtensorMap &mapX, const CUtenso
             if (warp == 12 && lane == 0) SSD_TRACE_EV(10, u);
             if (!STATE_ONLY && u >= 1) ok = epilogue(u - 1);
         }
-        // end of the segment: the state after the last token
+        // end of the segment: the state after the last token.  The full walk has waited for every
+        // earlier phase of h_ready[j], so the last one is the next to complete; the state-only walk
+        // has not (a parity wait more than one phase ahead would pass at once), so it waits for the
+        // state issuer's drain commit instead, which completes once, after the last state UMMA
         if (ok) {
             for (int j = 0; j < KH; ++j) {
-                ok = mbar_wait<kInlW>(&Bb.h_ready[j], (nblk - 1) & 1, abort);
+                ok = STATE_ONLY ? mbar_wait<kInlW>(&Bb.drain_s, 0, abort)
+                                : mbar_wait<kInlW>(&Bb.h_ready[j], (nblk - 1) & 1, abort);
                 if (!ok) break;
                 tc_fence_after();
                 const int h = it.h0 + j;

@@ -125,13 +125,16 @@ def _dev(inp, t0=None, t1=None):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("kind", ["tensor", "simt", "tensor_varlen", "simt_varlen"])
+@pytest.mark.parametrize("kind", ["tensor", "simt", "tensor_varlen", "simt_varlen", "tensor_short"])
 def test_summary_matches_oracle(kind):
-    """End state from a zero state and total log decay of every sequence."""
+    """End state from a zero state and total log decay of every sequence (tensor_short:
+    sequences of one and two 128-token blocks, where the end state is read right
+    after the last state update)."""
     import torch
     import mamba_ssd_layer_fwd_b200 as ssd
     from _helpers import small_inputs, record_parity
-    varlen = [300, 0, 129, 411] if kind.endswith("varlen") else None
+    varlen = {"tensor_varlen": [300, 0, 129, 411], "simt_varlen": [300, 0, 129, 411],
+              "tensor_short": [129, 1, 256, 129, 2]}.get(kind)
     inp = small_inputs(batch=2, seqlen=700, H=4, P=64, N=128, G=2, Q=256, init=False, varlen=varlen, seed=51)
     path = "tensor" if kind.startswith("tensor") else "simt"
     t = _dev(inp)
