@@ -372,7 +372,8 @@ class Forward:
         inp = self.inp
         alg_bytes = algorithmic_bytes(inp)
         peak, peak_kind = measured_peaks()
-        kernel = "ssd_tc_walk" if self.resolved == "tensor" else "chunk_scan_kernel"
+        # tensor path: the walk launches (ssd_tc_walk, and ssd_tc_fused for rows cut into segments)
+        kernel = "ssd_tc_walk+fused" if self.resolved == "tensor" else "chunk_scan_kernel"
         cm = statistics.median(comp_ms)
         mm = statistics.median(main_ms)
         achieved = alg_bytes / (cm * 1e-3) / 1e9
