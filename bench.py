@@ -654,6 +654,19 @@ def decode_bytes(inp: dict) -> int:
     return int(2 * b * H * P * N * 4 + (2 * b * H * P + b * H + 2 * b * G * N) * es)
 
 
+def run_backward(args):
+    """The backward sub-object alone (one GPU): `ssd_bwd` on the workload, with
+    the same timing and check as in the forward's JSON line."""
+    import torch
+    import mamba_ssd_layer_fwd_b200 as ssd
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    b = measure_backward(ssd, args, dev, flush, steps=args.steps)
+    print(json.dumps({"op": "backward", **(b or {"unavailable": "the workload is not bf16"})}))
+    return 0
+
+
 def run_decode(args):
     """One `ssd_decode_step` per step over every row of the decode workload
     (the state stays resident on the device, as in serving)."""
@@ -788,8 +801,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sub-workloads", action="store_true",
                     help="skip the per-workload measurements that follow the headline")
-    ap.add_argument("--op", choices=["fwd", "decode"], default="fwd",
-                    help="fwd: the chunked forward (default); decode: one recurrent step per row")
+    ap.add_argument("--op", choices=["fwd", "decode", "backward"], default="fwd",
+                    help="fwd: the chunked forward (default); decode: one recurrent step per row; "
+                         "backward: ssd_bwd alone on the workload (its sub-object, printed as one JSON line)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)      # at least 3 untimed warm-up steps
     if args.op == "decode" and args.workload == "mamba2_2p7b":
@@ -798,6 +812,8 @@ def main():
         return run_reference(args)
     if args.op == "decode":
         return run_decode(args)
+    if args.op == "backward":
+        return run_backward(args)
     return run_ours(args)
 
 

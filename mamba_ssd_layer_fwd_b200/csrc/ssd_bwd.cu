@@ -92,13 +92,24 @@ bwd_state_passing_kernel(Plan plan, Dims d, const float *__restrict__ cs, float 
     if (e >= PN) return;
     const SeqDesc sq = plan.seqs[s];
     float gv = dfinal ? dfinal[((size_t)s * d.H + h) * PN + e] : 0.0f;
-    for (int j = sq.nchunks - 1; j >= 0; --j) {
-        const int c = sq.chunk0 + j;
-        const size_t idx = ((size_t)c * d.H + h) * PN + e;
-        const float u = gbuf[idx];
-        gbuf[idx] = gv;
-        const float decay = __expf(cs[((size_t)c * d.H + h) * kBQ + kBQ - 1]);
-        gv = fmaf(decay, gv, u);
+    // loads in groups of chunks ahead of the chain (see state_passing_kernel)
+    constexpr int kGroup = 8;
+    for (int j0 = sq.nchunks - 1; j0 >= 0; j0 -= kGroup) {
+        float uv[kGroup], dk[kGroup];
+#pragma unroll
+        for (int i = 0; i < kGroup; ++i) {
+            const int c = sq.chunk0 + j0 - i;
+            const bool has = j0 - i >= 0;
+            uv[i] = has ? gbuf[((size_t)c * d.H + h) * PN + e] : 0.0f;
+            dk[i] = has ? __expf(cs[((size_t)c * d.H + h) * kBQ + kBQ - 1]) : 0.0f;
+        }
+#pragma unroll
+        for (int i = 0; i < kGroup; ++i) {
+            if (j0 - i >= 0) {
+                gbuf[((size_t)(sq.chunk0 + j0 - i) * d.H + h) * PN + e] = gv;
+                gv = fmaf(dk[i], gv, uv[i]);
+            }
+        }
     }
     if (dinit) dinit[((size_t)s * d.H + h) * PN + e] = gv;
 }
@@ -110,15 +121,22 @@ struct BwdArgs {
     float *dx, *ddt, *dA_log, *dB, *dC, *dD;
 };
 
+// Head-channel rows are padded to PA = P rounded up to 4 (zeros) plus 4, so that the
+// register-tiled products read them as float4.
 size_t chunk_smem_floats(int P, int N)
 {
-    const int PS = P + 1, NS = N + 1, QS = kBQ + 1;
+    const int PA = (P + 3) & ~3, PS = PA + 4, NS = N + 1, QS = kBQ + 1;
     return (size_t)2 * kBQ * NS        // B, C
            + 2 * kBQ * NS              // dB, dC accumulators
            + 2 * kBQ * PS              // x, dy
            + 3 * kBQ * QS              // C B^T, L, dy . x
-           + 2 * P * (kNT + 1)         // H_c, G_{c+1} tiles
+           + 2 * kNT * PS              // H_c, G_{c+1} tiles, transposed
            + 8 * kBQ + 32;             // per-token vectors, reductions
+}
+
+__device__ __forceinline__ float dot4(const float4 a, const float4 b, float acc)
+{
+    return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, fmaf(a.w, b.w, acc))));
 }
 
 template <typename T>
@@ -131,7 +149,7 @@ bwd_chunk_kernel(Plan plan, Dims d, BwdArgs a)
     const ChunkDesc ch = plan.chunks[c];
     const int g = blockIdx.y;
     const int P = d.P, N = d.N, H = d.H, G = d.G;
-    const int PS = P + 1, NS = N + 1, QS = kBQ + 1;
+    const int PA = (P + 3) & ~3, PG = PA / 4, PS = PA + 4, NS = N + 1, QS = kBQ + 1;
     const int len = ch.len;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     float *Bs = smem;                      // kBQ x NS
@@ -143,9 +161,9 @@ bwd_chunk_kernel(Plan plan, Dims d, BwdArgs a)
     float *CB = DYs + kBQ * PS;            // kBQ x QS: C_l . B_s
     float *Lm = CB + kBQ * QS;             // exp(cs_l - cs_s), s <= l < len
     float *DX = Lm + kBQ * QS;             // dy_l . x_s
-    float *Ht = DX + kBQ * QS;             // P x (kNT + 1)
-    float *Gt = Ht + P * (kNT + 1);
-    float *css = Gt + P * (kNT + 1);       // kBQ
+    float *Ht = DX + kBQ * QS;             // kNT x PS: Ht[nn][p] = H_c[p][n0 + nn]
+    float *Gt = Ht + kNT * PS;             // the same for G_{c+1}
+    float *css = Gt + kNT * PS;            // kBQ
     float *dls = css + kBQ;                // delta (0 past the chunk's end)
     float *fxs = dls + kBQ;                // x_s . (Gn B_s)
     float *dhc = fxs + kBQ;                // dy_l . (H C_l)
@@ -175,7 +193,14 @@ bwd_chunk_kernel(Plan plan, Dims d, BwdArgs a)
         CB[l * QS + s] = v;
     }
 
-    constexpr int kMaxOut = kBQ * 128 / kBThreads;   // (s, p) outputs per thread, P <= 128
+    // pad columns p in [P, PA) of the x, dy, H and G tiles: zero, never written again
+    for (int i = tid; i < (2 * kBQ + 2 * kNT) * (PA - P); i += kBThreads) {
+        const int r = i / (PA - P), p = P + i % (PA - P);
+        (r < 2 * kBQ ? Xs : Ht)[(r % (2 * kBQ)) * PS + p] = 0.0f;   // Xs, DYs and Ht, Gt are adjacent
+    }
+    // the dx terms are computed in (token pair, 4-channel group) items, at most two per thread
+    constexpr int kMaxItems = (kBQ / 2) * (128 / 4) / kBThreads;
+    const int n_items = (kBQ / 2) * PG;
     for (int h = g * d.heads_per_group; h < (g + 1) * d.heads_per_group; ++h) {
         const float A = -__expf(a.A_log[h]);
         const float Dh = a.D ? a.D[h] : 0.0f;
@@ -219,18 +244,30 @@ bwd_chunk_kernel(Plan plan, Dims d, BwdArgs a)
             for (int o = 16; o > 0; o >>= 1) dd += __shfl_xor_sync(0xffffffffu, dd, o);
             if (t == 0) red[1] = dd;
         }
-        // intra terms of dx (into registers), dB, dC
-        float dxr[kMaxOut];
+        // intra terms of dx (into registers): sum over l >= s of W[l, s] dy_l, W = L o CB (zero above
+        // the diagonal), two tokens by four channels per item
+        float dxa[kMaxItems][2][4], gba[kMaxItems][2][4];
 #pragma unroll
-        for (int k = 0; k < kMaxOut; ++k) {
-            const int i = tid + k * kBThreads;
-            float v = 0.0f;
-            if (i < kBQ * P) {
-                const int s = i / P, p = i % P;
-                for (int l = s; l < kBQ; ++l) v = fmaf(Lm[l * QS + s] * CB[l * QS + s], DYs[l * PS + p], v);
+        for (int k = 0; k < kMaxItems; ++k) {
+#pragma unroll
+            for (int a2 = 0; a2 < 2; ++a2)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) dxa[k][a2][i] = gba[k][a2][i] = 0.0f;
+            const int item = tid + k * kBThreads;
+            if (item < n_items) {
+                const int s0 = 2 * (item / PG), p0 = 4 * (item % PG);
+                for (int l = s0; l < kBQ; ++l) {
+                    const float w0 = Lm[l * QS + s0] * CB[l * QS + s0];
+                    const float w1 = Lm[l * QS + s0 + 1] * CB[l * QS + s0 + 1];
+                    const float4 y4 = *reinterpret_cast<const float4 *>(&DYs[l * PS + p0]);
+                    dxa[k][0][0] = fmaf(w0, y4.x, dxa[k][0][0]); dxa[k][0][1] = fmaf(w0, y4.y, dxa[k][0][1]);
+                    dxa[k][0][2] = fmaf(w0, y4.z, dxa[k][0][2]); dxa[k][0][3] = fmaf(w0, y4.w, dxa[k][0][3]);
+                    dxa[k][1][0] = fmaf(w1, y4.x, dxa[k][1][0]); dxa[k][1][1] = fmaf(w1, y4.y, dxa[k][1][1]);
+                    dxa[k][1][2] = fmaf(w1, y4.z, dxa[k][1][2]); dxa[k][1][3] = fmaf(w1, y4.w, dxa[k][1][3]);
+                }
             }
-            dxr[k] = v;
         }
+        // intra terms of dB, dC
         for (int i = tid; i < kBQ * N; i += kBThreads) {
             const int s = i / N, n = i % N;
             float vb = 0.0f, vc = 0.0f;
@@ -239,12 +276,9 @@ bwd_chunk_kernel(Plan plan, Dims d, BwdArgs a)
             dBs[s * NS + n] += dls[s] * vb;
             dCs[s * NS + n] += vc;
         }
-        // inter terms, over tiles of kNT dstate columns of H_c and G_{c+1}
+        // inter terms, over tiles of kNT dstate columns of H_c and G_{c+1} (stored transposed)
         const float *Hc = a.states + ((size_t)c * H + h) * (size_t)P * N;
         const float *Gn = a.gbuf + ((size_t)c * H + h) * (size_t)P * N;
-        float gbr[kMaxOut];
-#pragma unroll
-        for (int k = 0; k < kMaxOut; ++k) gbr[k] = 0.0f;
         float ghp = 0.0f;
         for (int n0 = 0; n0 < N; n0 += kNT) {
             const int nt = min(kNT, N - n0);
@@ -254,37 +288,77 @@ bwd_chunk_kernel(Plan plan, Dims d, BwdArgs a)
                 const bool v = nn < nt;
                 const float hv = v ? Hc[(size_t)p * N + n0 + nn] : 0.0f;
                 const float gv = v ? Gn[(size_t)p * N + n0 + nn] : 0.0f;
-                Ht[p * (kNT + 1) + nn] = hv;
-                Gt[p * (kNT + 1) + nn] = gv;
+                Ht[nn * PS + p] = hv;
+                Gt[nn * PS + p] = gv;
                 ghp = fmaf(hv, gv, ghp);
             }
             __syncthreads();
-            // (Gn B_s)[p] over this tile
+            // (Gn B_s)[p] over this tile, per (token pair, channel group) item
 #pragma unroll
-            for (int k = 0; k < kMaxOut; ++k) {
-                const int i = tid + k * kBThreads;
-                if (i < kBQ * P) {
-                    const int s = i / P, p = i % P;
-                    float v = gbr[k];
-                    for (int nn = 0; nn < nt; ++nn) v = fmaf(Bs[s * NS + n0 + nn], Gt[p * (kNT + 1) + nn], v);
-                    gbr[k] = v;
+            for (int k = 0; k < kMaxItems; ++k) {
+                const int item = tid + k * kBThreads;
+                if (item < n_items) {
+                    const int s0 = 2 * (item / PG), p0 = 4 * (item % PG);
+                    for (int nn = 0; nn < nt; ++nn) {
+                        const float b0 = Bs[s0 * NS + n0 + nn], b1 = Bs[(s0 + 1) * NS + n0 + nn];
+                        const float4 g4 = *reinterpret_cast<const float4 *>(&Gt[nn * PS + p0]);
+                        gba[k][0][0] = fmaf(b0, g4.x, gba[k][0][0]); gba[k][0][1] = fmaf(b0, g4.y, gba[k][0][1]);
+                        gba[k][0][2] = fmaf(b0, g4.z, gba[k][0][2]); gba[k][0][3] = fmaf(b0, g4.w, gba[k][0][3]);
+                        gba[k][1][0] = fmaf(b1, g4.x, gba[k][1][0]); gba[k][1][1] = fmaf(b1, g4.y, gba[k][1][1]);
+                        gba[k][1][2] = fmaf(b1, g4.z, gba[k][1][2]); gba[k][1][3] = fmaf(b1, g4.w, gba[k][1][3]);
+                    }
                 }
             }
-            // x_s . Gn[:, n] and dy_l . H[:, n] for the tile's columns
-            for (int i = tid; i < kBQ * kNT; i += kBThreads) {
-                const int s = i / kNT, nn = i % kNT;
-                if (nn >= nt) continue;
-                float xg = 0.0f, dh = 0.0f;
-                for (int p = 0; p < P; ++p) {
-                    xg = fmaf(Xs[s * PS + p], Gt[p * (kNT + 1) + nn], xg);
-                    dh = fmaf(DYs[s * PS + p], Ht[p * (kNT + 1) + nn], dh);
+            // x_s . Gn[:, n] and dy_s . H[:, n]: tokens s0, s0 + 1 by columns nn, nn + 16 per thread
+            {
+                const int s0 = 2 * (tid >> 4), nb = tid & 15;
+                float xg[2][2] = {{0.0f, 0.0f}, {0.0f, 0.0f}}, dh[2][2] = {{0.0f, 0.0f}, {0.0f, 0.0f}};
+                for (int p0 = 0; p0 < PA; p0 += 4) {
+                    const float4 xa = *reinterpret_cast<const float4 *>(&Xs[s0 * PS + p0]);
+                    const float4 xb = *reinterpret_cast<const float4 *>(&Xs[(s0 + 1) * PS + p0]);
+                    const float4 ya = *reinterpret_cast<const float4 *>(&DYs[s0 * PS + p0]);
+                    const float4 yb = *reinterpret_cast<const float4 *>(&DYs[(s0 + 1) * PS + p0]);
+                    const float4 g0 = *reinterpret_cast<const float4 *>(&Gt[nb * PS + p0]);
+                    const float4 g1 = *reinterpret_cast<const float4 *>(&Gt[(nb + 16) * PS + p0]);
+                    const float4 h0 = *reinterpret_cast<const float4 *>(&Ht[nb * PS + p0]);
+                    const float4 h1 = *reinterpret_cast<const float4 *>(&Ht[(nb + 16) * PS + p0]);
+                    xg[0][0] = dot4(xa, g0, xg[0][0]); xg[0][1] = dot4(xa, g1, xg[0][1]);
+                    xg[1][0] = dot4(xb, g0, xg[1][0]); xg[1][1] = dot4(xb, g1, xg[1][1]);
+                    dh[0][0] = dot4(ya, h0, dh[0][0]); dh[0][1] = dot4(ya, h1, dh[0][1]);
+                    dh[1][0] = dot4(yb, h0, dh[1][0]); dh[1][1] = dot4(yb, h1, dh[1][1]);
                 }
-                const int n = n0 + nn;
-                const float e2 = __expf(fminf(css[kBQ - 1] - css[s], 0.0f));
-                dBs[s * NS + n] += dls[s] * e2 * xg;
-                dCs[s * NS + n] += (s < len ? __expf(css[s]) : 0.0f) * dh;
-                atomicAdd(&fxs[s], xg * Bs[s * NS + n]);
-                atomicAdd(&dhc[s], dh * Cs[s * NS + n]);
+                float fx[2] = {0.0f, 0.0f}, dc[2] = {0.0f, 0.0f};
+#pragma unroll
+                for (int a2 = 0; a2 < 2; ++a2) {
+                    const int s = s0 + a2;
+                    const float e2 = __expf(fminf(css[kBQ - 1] - css[s], 0.0f));
+                    const float ec = s < len ? __expf(css[s]) : 0.0f;
+#pragma unroll
+                    for (int b2 = 0; b2 < 2; ++b2) {
+                        const int nn = nb + 16 * b2;
+                        if (nn < nt) {
+                            const int n = n0 + nn;
+                            dBs[s * NS + n] += dls[s] * e2 * xg[a2][b2];
+                            dCs[s * NS + n] += ec * dh[a2][b2];
+                            fx[a2] = fmaf(xg[a2][b2], Bs[s * NS + n], fx[a2]);
+                            dc[a2] = fmaf(dh[a2][b2], Cs[s * NS + n], dc[a2]);
+                        }
+                    }
+                }
+                // over the 16 lanes holding this token pair (lanes 16 t .. 16 t + 15 of the warp)
+#pragma unroll
+                for (int o = 8; o > 0; o >>= 1)
+#pragma unroll
+                    for (int a2 = 0; a2 < 2; ++a2) {
+                        fx[a2] += __shfl_xor_sync(0xffffffffu, fx[a2], o);
+                        dc[a2] += __shfl_xor_sync(0xffffffffu, dc[a2], o);
+                    }
+                if (nb == 0) {
+                    atomicAdd(&fxs[s0], fx[0]);
+                    atomicAdd(&fxs[s0 + 1], fx[1]);
+                    atomicAdd(&dhc[s0], dc[0]);
+                    atomicAdd(&dhc[s0 + 1], dc[1]);
+                }
             }
         }
         for (int o = 16; o > 0; o >>= 1) ghp += __shfl_xor_sync(0xffffffffu, ghp, o);
@@ -292,14 +366,21 @@ bwd_chunk_kernel(Plan plan, Dims d, BwdArgs a)
         __syncthreads();
         // dx = D dy + delta (intra + e2 Gn B)
 #pragma unroll
-        for (int k = 0; k < kMaxOut; ++k) {
-            const int i = tid + k * kBThreads;
-            if (i < kBQ * P) {
-                const int s = i / P, p = i % P;
-                if (s < len) {
-                    const float e2 = __expf(fminf(css[kBQ - 1] - css[s], 0.0f));
-                    a.dx[((size_t)(ch.tok0 + s) * H + h) * P + p] =
-                        fmaf(Dh, DYs[s * PS + p], dls[s] * (dxr[k] + e2 * gbr[k]));
+        for (int k = 0; k < kMaxItems; ++k) {
+            const int item = tid + k * kBThreads;
+            if (item < n_items) {
+                const int s0 = 2 * (item / PG), p0 = 4 * (item % PG);
+#pragma unroll
+                for (int a2 = 0; a2 < 2; ++a2) {
+                    const int s = s0 + a2;
+                    if (s < len) {
+                        const float e2 = __expf(fminf(css[kBQ - 1] - css[s], 0.0f));
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            if (p0 + i < P)
+                                a.dx[((size_t)(ch.tok0 + s) * H + h) * P + p0 + i] =
+                                    fmaf(Dh, DYs[s * PS + p0 + i], dls[s] * (dxa[k][a2][i] + e2 * gba[k][a2][i]));
+                    }
                 }
             }
         }

@@ -133,13 +133,26 @@ state_passing_kernel(Plan plan, Dims d, const float *__restrict__ cs, float *__r
     if (e >= PN) return;
     const SeqDesc sq = plan.seqs[s];
     float hv = init ? init[((size_t)s * d.H + h) * PN + e] : 0.0f;
-    for (int j = 0; j < sq.nchunks; ++j) {
-        const int c = sq.chunk0 + j;
-        const size_t idx = ((size_t)c * d.H + h) * PN + e;
-        const float sv = states[idx];
-        states[idx] = hv;                       // state entering chunk c
-        const float decay = __expf(cs[((size_t)c * d.H + h) * d.Q + d.Q - 1]);
-        hv = fmaf(decay, hv, sv);
+    // the chunks' states and decays are loaded in groups before the chain uses them, so the
+    // chain waits on memory once per group, not once per chunk
+    constexpr int kGroup = 8;
+    for (int j0 = 0; j0 < sq.nchunks; j0 += kGroup) {
+        float sv[kGroup], dk[kGroup];
+#pragma unroll
+        for (int i = 0; i < kGroup; ++i) {
+            const int c = sq.chunk0 + j0 + i;
+            const bool has = j0 + i < sq.nchunks;
+            sv[i] = has ? states[((size_t)c * d.H + h) * PN + e] : 0.0f;
+            dk[i] = has ? __expf(cs[((size_t)c * d.H + h) * d.Q + d.Q - 1]) : 0.0f;
+        }
+#pragma unroll
+        for (int i = 0; i < kGroup; ++i) {
+            if (j0 + i < sq.nchunks) {
+                const int c = sq.chunk0 + j0 + i;
+                states[((size_t)c * d.H + h) * PN + e] = hv;     // state entering chunk c
+                hv = fmaf(dk[i], hv, sv[i]);
+            }
+        }
     }
     if (final_states) final_states[((size_t)s * d.H + h) * PN + e] = hv;
 }

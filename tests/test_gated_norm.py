@@ -56,6 +56,17 @@ def test_gated_norm_tensor_path_ragged(N, G, H):
     check_gated(inp, f"tensor ragged N={N}", path="tensor", seed=1)
 
 
+@pytest.mark.parametrize("N", [128, 256])
+def test_gated_norm_single_launch_segmented(N):
+    """Equal-length rows cut into segments: the gated norm in the epilogue of the
+    segmented walk's second (full) walk."""
+    import mamba_ssd_layer_fwd_b200 as ssd
+    inp = small_inputs(batch=1, seqlen=3000, H=2, P=64, N=N, G=1, Q=256, init=True, seed=65 + N)
+    t = to_device(inp)
+    assert ssd.launch_count(ssd.params_for(t["x"], t["B"], 256, None, True, "tensor")) == 1
+    check_gated(inp, f"tensor single-launch segmented N={N}", path="tensor", seed=3)
+
+
 def test_gated_norm_tensor_path_segmented_varlen():
     inp = small_inputs(H=2, P=64, N=128, G=1, Q=256, varlen=[6000, 0, 129, 3000], init=True, seed=61)
     check_gated(inp, "tensor packed, segmented", path="tensor", seed=2, bias=False)
