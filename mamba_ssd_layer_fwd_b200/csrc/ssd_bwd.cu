@@ -44,7 +44,9 @@ __device__ __forceinline__ float sigmoid_f32(float r)
     return r >= 0.0f ? 1.0f / (1.0f + e) : e / (1.0f + e);
 }
 
-// U_c[p][n] = sum_l exp(cs_l) dy_l[p] C_l[n], written into `ubuf` (the layout of the chunk states)
+// U_c[p][n] = sum_l exp(cs_l) dy_l[p] C_l[n], written into `ubuf` (the layout of the chunk states).
+// Rows of the shared tiles are padded to a multiple of 4 (zeros); each thread accumulates a
+// 4 x 4 register tile (four channels by four state columns) from float4 rows.
 template <typename T>
 __global__ void __launch_bounds__(kBThreads)
 bwd_dstate_kernel(Plan plan, Dims d, const T *__restrict__ dy, const T *__restrict__ Cm,
@@ -56,26 +58,50 @@ bwd_dstate_kernel(Plan plan, Dims d, const T *__restrict__ dy, const T *__restri
     const ChunkDesc ch = plan.chunks[c];
     const int h = blockIdx.y, g = h / d.heads_per_group;
     const int P = d.P, N = d.N;
-    float *Ys = smem;                 // kBQ x P (weighted dy)
-    float *Cs = Ys + kBQ * P;         // kBQ x N
+    const int PA = (P + 3) & ~3, NA = (N + 3) & ~3;
+    float *Ys = smem;                 // kBQ x PA (weighted dy)
+    float *Cs = Ys + kBQ * PA;        // kBQ x NA
     const float *csc = cs + ((size_t)c * d.H + h) * kBQ;
-    for (int i = threadIdx.x; i < kBQ * P; i += kBThreads) {
-        const int l = i / P, p = i % P;
-        Ys[i] = l < ch.len ? __expf(csc[l]) * to_f32(dy[((size_t)(ch.tok0 + l) * d.H + h) * P + p]) : 0.0f;
+    for (int i = threadIdx.x; i < kBQ * PA; i += kBThreads) {
+        const int l = i / PA, p = i % PA;
+        Ys[i] = l < ch.len && p < P ? __expf(csc[l]) * to_f32(dy[((size_t)(ch.tok0 + l) * d.H + h) * P + p]) : 0.0f;
     }
-    for (int i = threadIdx.x; i < kBQ * N; i += kBThreads) {
-        const int l = i / N, n = i % N;
-        Cs[i] = l < ch.len ? to_f32(Cm[((size_t)(ch.tok0 + l) * d.G + g) * N + n]) : 0.0f;
+    for (int i = threadIdx.x; i < kBQ * NA; i += kBThreads) {
+        const int l = i / NA, n = i % NA;
+        Cs[i] = l < ch.len && n < N ? to_f32(Cm[((size_t)(ch.tok0 + l) * d.G + g) * N + n]) : 0.0f;
     }
     __syncthreads();
-    const int PN = P * N;
-    float *out = ubuf + ((size_t)c * d.H + h) * PN;
-    for (int e = threadIdx.x; e < PN; e += kBThreads) {
-        const int p = e / N, n = e % N;
-        float a = 0.0f;
-#pragma unroll 8
-        for (int l = 0; l < kBQ; ++l) a = fmaf(Ys[l * P + p], Cs[l * N + n], a);
-        out[e] = a;
+    const int NG = NA / 4, items = (PA / 4) * NG;
+    float *out = ubuf + ((size_t)c * d.H + h) * (size_t)P * N;
+    for (int it = threadIdx.x; it < items; it += kBThreads) {
+        const int p0 = 4 * (it / NG), n0 = 4 * (it % NG);
+        float acc[4][4];
+#pragma unroll
+        for (int a2 = 0; a2 < 4; ++a2)
+#pragma unroll
+            for (int b2 = 0; b2 < 4; ++b2) acc[a2][b2] = 0.0f;
+#pragma unroll 4
+        for (int l = 0; l < kBQ; ++l) {
+            const float4 y4 = *reinterpret_cast<const float4 *>(&Ys[l * PA + p0]);
+            const float4 c4 = *reinterpret_cast<const float4 *>(&Cs[l * NA + n0]);
+            const float yv[4] = {y4.x, y4.y, y4.z, y4.w}, cv[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+            for (int a2 = 0; a2 < 4; ++a2)
+#pragma unroll
+                for (int b2 = 0; b2 < 4; ++b2) acc[a2][b2] = fmaf(yv[a2], cv[b2], acc[a2][b2]);
+        }
+#pragma unroll
+        for (int a2 = 0; a2 < 4; ++a2) {
+            if (p0 + a2 >= P) break;
+            float *row = out + (size_t)(p0 + a2) * N + n0;
+            if (n0 + 4 <= N && (N & 3) == 0) {
+                *reinterpret_cast<float4 *>(row) = make_float4(acc[a2][0], acc[a2][1], acc[a2][2], acc[a2][3]);
+            } else {
+#pragma unroll
+                for (int b2 = 0; b2 < 4; ++b2)
+                    if (n0 + b2 < N) row[b2] = acc[a2][b2];
+            }
+        }
     }
 }
 
@@ -160,7 +186,7 @@ bwd_chunk_kernel(Plan plan, Dims d, BwdArgs a)
     float *DYs = Xs + kBQ * PS;
     float *CB = DYs + kBQ * PS;            // kBQ x QS: C_l . B_s
     float *Lm = CB + kBQ * QS;             // exp(cs_l - cs_s), s <= l < len
-    float *DX = Lm + kBQ * QS;             // dy_l . x_s
+    float *DX = Lm + kBQ * QS;             // M = L o (dy . x): L[l, s] (dy_l . x_s)
     float *Ht = DX + kBQ * QS;             // kNT x PS: Ht[nn][p] = H_c[p][n0 + nn]
     float *Gt = Ht + kNT * PS;             // the same for G_{c+1}
     float *css = Gt + kNT * PS;            // kBQ
@@ -226,8 +252,9 @@ bwd_chunk_kernel(Plan plan, Dims d, BwdArgs a)
             const int l = i / kBQ, s = i % kBQ;
             float v = 0.0f;
             for (int p = 0; p < P; ++p) v = fmaf(DYs[l * PS + p], Xs[s * PS + p], v);
-            DX[l * QS + s] = v;
-            Lm[l * QS + s] = (s <= l && l < len) ? __expf(fminf(css[l] - css[s], 0.0f)) : 0.0f;
+            const float lm = (s <= l && l < len) ? __expf(fminf(css[l] - css[s], 0.0f)) : 0.0f;
+            Lm[l * QS + s] = lm;
+            DX[l * QS + s] = lm * v;
         }
         __syncthreads();
         // per token: row and column sums of E and of W o (dy . x); dD.  The sums for d(cs)
@@ -236,11 +263,11 @@ bwd_chunk_kernel(Plan plan, Dims d, BwdArgs a)
         if (tid < kBQ) {
             const int t = tid;
             float row = 0.0f, col = 0.0f;
-            for (int s = 0; s < t; ++s) row = fmaf(Lm[t * QS + s] * CB[t * QS + s] * DX[t * QS + s], dls[s], row);
-            for (int l = t + 1; l < kBQ; ++l) col = fmaf(Lm[l * QS + t] * CB[l * QS + t], DX[l * QS + t], col);
+            for (int s = 0; s < t; ++s) row = fmaf(CB[t * QS + s] * DX[t * QS + s], dls[s], row);
+            for (int l = t + 1; l < kBQ; ++l) col = fmaf(CB[l * QS + t], DX[l * QS + t], col);
             rowv[t] = row;
             colv[t] = col;
-            float dd = t < len ? DX[t * QS + t] : 0.0f;
+            float dd = t < len ? DX[t * QS + t] : 0.0f;       // L[t, t] = 1
             for (int o = 16; o > 0; o >>= 1) dd += __shfl_xor_sync(0xffffffffu, dd, o);
             if (t == 0) red[1] = dd;
         }
@@ -268,13 +295,46 @@ bwd_chunk_kernel(Plan plan, Dims d, BwdArgs a)
             }
         }
         // intra terms of dB, dC
-        for (int i = tid; i < kBQ * N; i += kBThreads) {
-            const int s = i / N, n = i % N;
-            float vb = 0.0f, vc = 0.0f;
-            for (int l = s; l < kBQ; ++l) vb = fmaf(Lm[l * QS + s] * DX[l * QS + s], Cs[l * NS + n], vb);
-            for (int t = 0; t <= s; ++t) vc = fmaf(Lm[s * QS + t] * DX[s * QS + t] * dls[t], Bs[t * NS + n], vc);
-            dBs[s * NS + n] += dls[s] * vb;
-            dCs[s * NS + n] += vc;
+        // dB_s += delta_s sum_{l >= s} M[l, s] C_l and dC_s += sum_{t <= s} M[s, t] delta_t B_t
+        // (M zero above the diagonal): two tokens by four state columns nq + NQ k per item, so
+        // that the lanes of a warp read consecutive columns
+        const int NQ = (N + 3) / 4;
+        for (int it = tid; it < (kBQ / 2) * NQ; it += kBThreads) {
+            const int s0 = 2 * (it / NQ), nq = it % NQ;
+            float vb[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
+            float vc[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
+            for (int l = s0; l < kBQ; ++l) {
+                const float m0 = DX[l * QS + s0], m1 = DX[l * QS + s0 + 1];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int n = nq + NQ * k;
+                    const float cv = n < N ? Cs[l * NS + n] : 0.0f;
+                    vb[0][k] = fmaf(m0, cv, vb[0][k]);
+                    vb[1][k] = fmaf(m1, cv, vb[1][k]);
+                }
+            }
+            for (int t = 0; t <= s0 + 1; ++t) {
+                const float q0 = DX[s0 * QS + t] * dls[t], q1 = DX[(s0 + 1) * QS + t] * dls[t];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int n = nq + NQ * k;
+                    const float bv = n < N ? Bs[t * NS + n] : 0.0f;
+                    vc[0][k] = fmaf(q0, bv, vc[0][k]);
+                    vc[1][k] = fmaf(q1, bv, vc[1][k]);
+                }
+            }
+#pragma unroll
+            for (int a2 = 0; a2 < 2; ++a2) {
+                const int s = s0 + a2;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int n = nq + NQ * k;
+                    if (n < N) {
+                        dBs[s * NS + n] += dls[s] * vb[a2][k];
+                        dCs[s * NS + n] += vc[a2][k];
+                    }
+                }
+            }
         }
         // inter terms, over tiles of kNT dstate columns of H_c and G_{c+1} (stored transposed)
         const float *Hc = a.states + ((size_t)c * H + h) * (size_t)P * N;
@@ -392,7 +452,7 @@ bwd_chunk_kernel(Plan plan, Dims d, BwdArgs a)
             float Fsum = F;
             for (int o = 16; o > 0; o >>= 1) Fsum += __shfl_xor_sync(0xffffffffu, Fsum, o);
             float dcs = rowv[t] - dls[t] * colv[t] + (t < len ? __expf(css[t]) : 0.0f) * dhc[t] - F;
-            const float colx = colv[t] + Lm[t * QS + t] * CB[t * QS + t] * DX[t * QS + t];   // with the diagonal
+            const float colx = colv[t] + CB[t * QS + t] * DX[t * QS + t];   // with the diagonal
             if (t == kBQ - 1) dcs += Fsum + __expf(css[kBQ - 1]) * red[0];
             // reverse inclusive scan: ddA_k = sum_{l >= k} dcs_l
             float v = dcs;
@@ -454,7 +514,7 @@ cudaError_t launch_bwd(const Plan &plan, const Dims &d, const SimtArgs &fa, cons
     const int PN = d.P * d.N;
     if (plan.max_chunks > 0) {
         const dim3 gc(plan.max_chunks, d.H);
-        const size_t sd = sizeof(float) * kBQ * (d.P + d.N);
+        const size_t sd = sizeof(float) * kBQ * (((d.P + 3) & ~3) + ((d.N + 3) & ~3));
         if (bf16) {
             e = cudaFuncSetAttribute(bwd_dstate_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sd);
             if (e != cudaSuccess) return e;

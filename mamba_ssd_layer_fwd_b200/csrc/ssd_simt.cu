@@ -58,7 +58,10 @@ chunk_cumsum_kernel(Plan plan, Dims d, const T *__restrict__ dt, const float *__
 }
 
 // -------------------------------------------------------------- chunk_state
-constexpr int kStateEPT = 16;   // outputs per thread per pass
+// Register tiles: each thread accumulates 4 x 4 outputs (four channels by four state columns)
+// per item, at most two items at a time, from float4 rows of the shared tiles (rows padded to a
+// multiple of 4 with zeros).
+constexpr int kStateItems = 2;   // items per thread per pass
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
@@ -73,9 +76,10 @@ chunk_state_kernel(Plan plan, Dims d, const T *__restrict__ x, const T *__restri
     const int h = blockIdx.y;
     const int g = h / d.heads_per_group;
     const int P = d.P, N = d.N, Q = d.Q;
-    float *Xs = smem;                       // kTile x P   (weighted x)
-    float *Bs = Xs + kTile * P;             // kTile x N
-    float *w = Bs + kTile * N;              // Q
+    const int PA = (P + 3) & ~3, NA = (N + 3) & ~3;
+    float *Xs = smem;                       // kTile x PA (weighted x)
+    float *Bs = Xs + kTile * PA;            // kTile x NA
+    float *w = Bs + kTile * NA;             // Q
     const float *csc = cs + ((size_t)c * d.H + h) * Q;
     const float *dvc = dv + ((size_t)c * d.H + h) * Q;
     const float cs_last = csc[Q - 1];
@@ -83,40 +87,64 @@ chunk_state_kernel(Plan plan, Dims d, const T *__restrict__ x, const T *__restri
         w[l] = l < ch.len ? __expf(fminf(cs_last - csc[l], 0.0f)) * dvc[l] : 0.0f;   // <= 0 up to rounding
     __syncthreads();
 
-    const int PN = P * N;
-    float *out = states + ((size_t)c * d.H + h) * PN;
-    for (int e0 = 0; e0 < PN; e0 += kThreads * kStateEPT) {
-        float acc[kStateEPT];
+    const int NG = NA / 4, items = (PA / 4) * NG;
+    float *out = states + ((size_t)c * d.H + h) * (size_t)P * N;
+    for (int b0 = 0; b0 < items; b0 += kThreads * kStateItems) {
+        float acc[kStateItems][4][4];
 #pragma unroll
-        for (int i = 0; i < kStateEPT; ++i) acc[i] = 0.0f;
+        for (int k = 0; k < kStateItems; ++k)
+#pragma unroll
+            for (int a2 = 0; a2 < 4; ++a2)
+#pragma unroll
+                for (int b2 = 0; b2 < 4; ++b2) acc[k][a2][b2] = 0.0f;
         for (int l0 = 0; l0 < ch.len; l0 += kTile) {
-            for (int i = threadIdx.x; i < kTile * P; i += kThreads) {
-                const int r = i / P, p = i % P;
+            for (int i = threadIdx.x; i < kTile * PA; i += kThreads) {
+                const int r = i / PA, p = i % PA;
                 const int l = l0 + r;
-                Xs[i] = l < ch.len ? w[l] * to_f32(x[((size_t)(ch.tok0 + l) * d.H + h) * P + p]) : 0.0f;
+                Xs[i] = l < ch.len && p < P ? w[l] * to_f32(x[((size_t)(ch.tok0 + l) * d.H + h) * P + p]) : 0.0f;
             }
-            for (int i = threadIdx.x; i < kTile * N; i += kThreads) {
-                const int r = i / N, n = i % N;
+            for (int i = threadIdx.x; i < kTile * NA; i += kThreads) {
+                const int r = i / NA, n = i % NA;
                 const int l = l0 + r;
-                Bs[i] = l < ch.len ? to_f32(Bm[((size_t)(ch.tok0 + l) * d.G + g) * N + n]) : 0.0f;
+                Bs[i] = l < ch.len && n < N ? to_f32(Bm[((size_t)(ch.tok0 + l) * d.G + g) * N + n]) : 0.0f;
             }
             __syncthreads();
 #pragma unroll
-            for (int i = 0; i < kStateEPT; ++i) {
-                const int e = e0 + threadIdx.x + i * kThreads;
-                if (e < PN) {
-                    const int p = e / N, n = e % N;
-                    float a = acc[i];
-                    for (int j = 0; j < kTile; ++j) a = fmaf(Xs[j * P + p], Bs[j * N + n], a);
-                    acc[i] = a;
+            for (int k = 0; k < kStateItems; ++k) {
+                const int it = b0 + threadIdx.x + k * kThreads;
+                if (it < items) {
+                    const int p0 = 4 * (it / NG), n0 = 4 * (it % NG);
+#pragma unroll 4
+                    for (int j = 0; j < kTile; ++j) {
+                        const float4 x4 = *reinterpret_cast<const float4 *>(&Xs[j * PA + p0]);
+                        const float4 b4 = *reinterpret_cast<const float4 *>(&Bs[j * NA + n0]);
+                        const float xv[4] = {x4.x, x4.y, x4.z, x4.w}, bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+                        for (int a2 = 0; a2 < 4; ++a2)
+#pragma unroll
+                            for (int b2 = 0; b2 < 4; ++b2) acc[k][a2][b2] = fmaf(xv[a2], bv[b2], acc[k][a2][b2]);
+                    }
                 }
             }
             __syncthreads();
         }
 #pragma unroll
-        for (int i = 0; i < kStateEPT; ++i) {
-            const int e = e0 + threadIdx.x + i * kThreads;
-            if (e < PN) out[e] = acc[i];
+        for (int k = 0; k < kStateItems; ++k) {
+            const int it = b0 + threadIdx.x + k * kThreads;
+            if (it >= items) continue;
+            const int p0 = 4 * (it / NG), n0 = 4 * (it % NG);
+#pragma unroll
+            for (int a2 = 0; a2 < 4; ++a2) {
+                if (p0 + a2 >= P) break;
+                float *row = out + (size_t)(p0 + a2) * N + n0;
+                if (n0 + 4 <= N && (N & 3) == 0) {
+                    *reinterpret_cast<float4 *>(row) = make_float4(acc[k][a2][0], acc[k][a2][1], acc[k][a2][2], acc[k][a2][3]);
+                } else {
+#pragma unroll
+                    for (int b2 = 0; b2 < 4; ++b2)
+                        if (n0 + b2 < N) row[b2] = acc[k][a2][b2];
+                }
+            }
         }
     }
 }
@@ -287,7 +315,10 @@ chunk_scan_kernel(Plan plan, Dims d, const T *__restrict__ x, const T *__restric
     }
 }
 
-size_t state_smem(const Dims &d) { return sizeof(float) * (kTile * d.P + kTile * d.N + d.Q); }
+size_t state_smem(const Dims &d)
+{
+    return sizeof(float) * (kTile * ((d.P + 3) & ~3) + kTile * ((d.N + 3) & ~3) + d.Q);
+}
 size_t scan_smem(const Dims &d)
 {
     return sizeof(float) * (2 * kTile * (d.N + 1) + 2 * kTile * (d.P + 1) + kTile * (kTile + 1) + 3 * kTile);
