@@ -79,14 +79,17 @@ def _code_only(text: str) -> str:
     return " ".join(text.split())
 
 
+# the sources of the tensor-core forward kernels, whose DRAM traffic profiles/traffic.json records
+TC_SOURCES = ("ssd_common.cuh", "ssd_tc.cu", "ssd_tc.cuh", "ssd_tc_prims.cuh")
+
+
 def kernel_source_hash() -> str:
-    """Hash of the library's CUDA sources (code only): the committed ncu
-    traffic figures apply while it matches."""
+    """Hash of the tensor-core forward kernels' CUDA sources (code only): the
+    committed ncu traffic figures apply while it matches."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mamba_ssd_layer_fwd_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".cuh")):
-            h.update(fn.encode() + b"\0" + _code_only(open(os.path.join(csrc, fn)).read()).encode() + b"\0")
+    for fn in TC_SOURCES:
+        h.update(fn.encode() + b"\0" + _code_only(open(os.path.join(csrc, fn)).read()).encode() + b"\0")
     return h.hexdigest()[:16]
 
 

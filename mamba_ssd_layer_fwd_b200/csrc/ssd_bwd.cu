@@ -36,6 +36,8 @@ namespace {
 constexpr int kBQ = 32;         // chunk length of the backward
 constexpr int kBThreads = 256;
 constexpr int kNT = 32;         // dstate columns per tile of H_c and G_{c+1}
+// the chunk kernel's register tiles map 256 threads onto 32 x 32 token pairs and token x column tiles
+static_assert(kBQ == 32 && kNT == 32 && kBThreads == 256, "the chunk kernel's thread mappings assume these sizes");
 
 __device__ __forceinline__ float sigmoid_f32(float r)
 {
@@ -248,13 +250,28 @@ bwd_chunk_kernel(Plan plan, Dims d, BwdArgs a)
         }
         if (tid < 2) red[tid] = 0.0f;
         __syncthreads();
-        for (int i = tid; i < kBQ * kBQ; i += kBThreads) {
-            const int l = i / kBQ, s = i % kBQ;
-            float v = 0.0f;
-            for (int p = 0; p < P; ++p) v = fmaf(DYs[l * PS + p], Xs[s * PS + p], v);
-            const float lm = (s <= l && l < len) ? __expf(fminf(css[l] - css[s], 0.0f)) : 0.0f;
-            Lm[l * QS + s] = lm;
-            DX[l * QS + s] = lm * v;
+        // dy_l . x_s for tokens l, l + 16 by s, s + 16 per thread (float4 rows; the lanes of a
+        // warp read rows 17 float4 apart, which fall in distinct bank groups)
+        {
+            const int l0 = tid >> 4, s0 = tid & 15;
+            float v[2][2] = {{0.0f, 0.0f}, {0.0f, 0.0f}};
+            for (int p0 = 0; p0 < PA; p0 += 4) {
+                const float4 ya = *reinterpret_cast<const float4 *>(&DYs[l0 * PS + p0]);
+                const float4 yb = *reinterpret_cast<const float4 *>(&DYs[(l0 + 16) * PS + p0]);
+                const float4 xa = *reinterpret_cast<const float4 *>(&Xs[s0 * PS + p0]);
+                const float4 xb = *reinterpret_cast<const float4 *>(&Xs[(s0 + 16) * PS + p0]);
+                v[0][0] = dot4(ya, xa, v[0][0]); v[0][1] = dot4(ya, xb, v[0][1]);
+                v[1][0] = dot4(yb, xa, v[1][0]); v[1][1] = dot4(yb, xb, v[1][1]);
+            }
+#pragma unroll
+            for (int a2 = 0; a2 < 2; ++a2)
+#pragma unroll
+                for (int b2 = 0; b2 < 2; ++b2) {
+                    const int l = l0 + 16 * a2, s = s0 + 16 * b2;
+                    const float lm = (s <= l && l < len) ? __expf(fminf(css[l] - css[s], 0.0f)) : 0.0f;
+                    Lm[l * QS + s] = lm;
+                    DX[l * QS + s] = lm * v[a2][b2];
+                }
         }
         __syncthreads();
         // per token: row and column sums of E and of W o (dy . x); dD.  The sums for d(cs)
