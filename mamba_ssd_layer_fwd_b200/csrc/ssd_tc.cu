@@ -905,13 +905,15 @@ __device__ __forceinline__ void walk_body(const CUtensorMap &mapX, const CUtenso
 #pragma unroll
             for (int mt = 0; mt < kMT; ++mt) {
                 const int n = kMT > 1 ? t + 128 * mt : t % N;   // N = 64: lanes 64..127 mirror 0..63
+                // all 64 loads of the row in flight before the first tensor-memory store (the
+                // stores are ordered after earlier loads, so a batch of 16 would wait 4 times)
+                uint32_t r[kP];
 #pragma unroll
-                for (int p0 = 0; p0 < kP; p0 += 16) {
-                    uint32_t r[16];
+                for (int p = 0; p < kP; ++p) r[p] = src ? __float_as_uint(src[(size_t)p * N + n]) : 0u;
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) r[i] = src ? __float_as_uint(src[(size_t)(p0 + i) * N + n]) : 0u;
-                    tmem_st16(tb + lane_base + kColH + 64 * (j + KH * mt) + p0, r);
-                }
+                for (int p0 = 0; p0 < kP; p0 += 16)
+                    tmem_st16(tb + lane_base + kColH + 64 * (j + KH * mt) + p0,
+                              *reinterpret_cast<uint32_t(*)[16]>(&r[p0]));
             }
         }
         tmem_st_wait();
