@@ -67,6 +67,16 @@ def test_gated_norm_single_launch_segmented(N):
     check_gated(inp, f"tensor single-launch segmented N={N}", path="tensor", seed=3)
 
 
+def test_gated_norm_one_head_items_and_tail():
+    """Odd heads per group (one-head items), and 160 two-head items on 148 SMs
+    (whole waves of two-head items, the rest as one-head items in a second,
+    overlapping launch), each with the gated norm in the epilogue."""
+    inp = small_inputs(batch=2, seqlen=300, H=3, P=64, N=128, G=1, Q=256, init=True, seed=66)
+    check_gated(inp, "tensor one-head items", path="tensor", seed=4)
+    inp = small_inputs(batch=2, seqlen=300, H=160, P=64, N=64, G=1, Q=256, init=True, seed=67)
+    check_gated(inp, "tensor two-head waves + one-head tail", path="tensor", seed=5)
+
+
 def test_gated_norm_tensor_path_segmented_varlen():
     inp = small_inputs(H=2, P=64, N=128, G=1, Q=256, varlen=[6000, 0, 129, 3000], init=True, seed=61)
     check_gated(inp, "tensor packed, segmented", path="tensor", seed=2, bias=False)
