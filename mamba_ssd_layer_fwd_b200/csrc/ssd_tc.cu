@@ -37,15 +37,16 @@
 // each other.  Every mbarrier wait is bounded (2 s); on a timeout the CTA
 // records SSD_ERR_TIMEOUT in the status word, drains, frees TMEM and exits.
 //
-// Equal-length rows that need no cuts take their work item from the block
-// index (no planner kernel); two-head items left over after whole waves of
-// the SMs run as one-head items in a second launch.  When there are too few
-// (sequence, head block) pairs to fill the GPU, each sequence is cut into
-// segments.  A first launch of the same kernel in state-only mode computes
-// every non-final segment's end state from zero;
-// a scan kernel turns those into each segment's entering state; the full
-// walk then starts every segment from its true state (Sec. 8.2: state
-// passing between pieces of a sequence).
+// Equal-length rows take their work item from the block index (no planner
+// kernel): whole waves of the SMs walk whole rows; the pairs left over run as
+// one-head items in a second launch, or (rows of many blocks, or fewer pairs
+// than SMs) are cut into segments and run by ssd_tc_fused, in which each
+// segment's CTA computes its end state from zero (state-only walk), the CTAs
+// of a pair chain the segment states between them, and every CTA then walks
+// its segment from its true entering state (Sec. 8.2: state passing between
+// pieces of a sequence).  Packed sequences take items from a planner kernel;
+// when they must be cut, a state-only launch, a scan kernel and the full walk
+// do the same in three launches.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
