@@ -168,7 +168,7 @@ __device__ __forceinline__ float dot4(const float4 a, const float4 b, float acc)
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kBThreads)
+__global__ void __launch_bounds__(kBThreads, 2)   // two CTAs per SM (registers and shared memory)
 bwd_chunk_kernel(Plan plan, Dims d, BwdArgs a)
 {
     extern __shared__ float smem[];
@@ -357,18 +357,34 @@ bwd_chunk_kernel(Plan plan, Dims d, BwdArgs a)
         const float *Hc = a.states + ((size_t)c * H + h) * (size_t)P * N;
         const float *Gn = a.gbuf + ((size_t)c * H + h) * (size_t)P * N;
         float ghp = 0.0f;
+        // each tile is fetched into registers one tile ahead, so its global loads are in flight
+        // while the previous tile's products run
+        constexpr int kTL = 128 * kNT / kBThreads;     // tile elements per thread (P <= 128)
+        float hn[kTL], gn[kTL];
+        auto fetch = [&](int t0) {
+            const int tn = min(kNT, N - t0);
+#pragma unroll
+            for (int k = 0; k < kTL; ++k) {
+                const int i = tid + k * kBThreads, p = i / kNT, nn = i % kNT;
+                const bool v = i < P * kNT && nn < tn;
+                hn[k] = v ? Hc[(size_t)p * N + t0 + nn] : 0.0f;
+                gn[k] = v ? Gn[(size_t)p * N + t0 + nn] : 0.0f;
+            }
+        };
+        fetch(0);
         for (int n0 = 0; n0 < N; n0 += kNT) {
             const int nt = min(kNT, N - n0);
             __syncthreads();
-            for (int i = tid; i < P * kNT; i += kBThreads) {
-                const int p = i / kNT, nn = i % kNT;
-                const bool v = nn < nt;
-                const float hv = v ? Hc[(size_t)p * N + n0 + nn] : 0.0f;
-                const float gv = v ? Gn[(size_t)p * N + n0 + nn] : 0.0f;
-                Ht[nn * PS + p] = hv;
-                Gt[nn * PS + p] = gv;
-                ghp = fmaf(hv, gv, ghp);
+#pragma unroll
+            for (int k = 0; k < kTL; ++k) {
+                const int i = tid + k * kBThreads, p = i / kNT, nn = i % kNT;
+                if (i < P * kNT) {
+                    Ht[nn * PS + p] = hn[k];
+                    Gt[nn * PS + p] = gn[k];
+                    ghp = fmaf(hn[k], gn[k], ghp);
+                }
             }
+            if (n0 + kNT < N) fetch(n0 + kNT);
             __syncthreads();
             // (Gn B_s)[p] over this tile, per (token pair, channel group) item
 #pragma unroll
