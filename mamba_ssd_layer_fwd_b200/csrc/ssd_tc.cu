@@ -1893,10 +1893,10 @@ cudaError_t launch_tc_uniform(const ssd_fwd_params &p, const Plan &plan, const T
 {
     const UniformPlan u = uniform_plan(p, s);
     const long long tokens = (long long)p.batch * p.seqlen;
-    // the status word, and the segmented launch's counters (one pair each)
+    // the status word, and the segmented launch's counters (two per pair, in the status region)
+    if (2 * (size_t)u.pairs > kStatusRegion / sizeof(int) - kSyncOffsetInts) return cudaErrorInvalidValue;
     cudaError_t e = cudaMemsetAsync(plan.status, 0, sizeof(int) * (kSyncOffsetInts + 2 * (size_t)u.pairs), stream);
     if (e != cudaSuccess || tokens == 0) return e;
-    if (2 * (size_t)u.pairs > kStatusRegion / sizeof(int) - kSyncOffsetInts) return cudaErrorInvalidValue;
     CUtensorMap mX, mB, mC, mY;
     // y has x's layout; its map moves 32-row slabs (one per epilogue warp)
     if (!make_map(&mX, a.x, (uint64_t)p.nheads * kP, (uint64_t)tokens) ||
