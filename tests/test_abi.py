@@ -148,6 +148,14 @@ def test_tensor_path_work_split(lib):
     assert ssd.launch_count(_tc_params(1, 32768, 48, 128, num_seqs=16)) == 2
     assert ssd.launch_count(_tc_params(1, 32768, 48, 128, num_seqs=1)) == 4
     assert ssd.launch_count(_tc_params(1, 512, 48, 128, num_seqs=4)) == 2
+    # the segmented launches keep their segment states in the workspace: 16 pairs x 9 segments
+    # x 2 heads x 64 x 256 fp32 for the 16K row; the 4 pairs left over after a whole wave of
+    # 148 rows of 32 blocks are cut into 32 segments; the one-head tail needs none
+    seg16k = 16 * 9 * 2 * 64 * 256 * 4
+    assert ssd.workspace_size(_tc_params(1, 16384, 32, 256, ngroups=8)) >= seg16k
+    assert ssd.launch_count(_tc_params(4, 4096, 76, 64)) == 2
+    assert ssd.workspace_size(_tc_params(4, 4096, 76, 64)) >= 4 * 32 * 2 * 64 * 64 * 4
+    assert ssd.workspace_size(_tc_params(8, 2048, 80, 128)) < 64 * 1024
     for p in (_tc_params(8, 2048, 80, 128), _tc_params(1, 16384, 32, 256, ngroups=8),
               _tc_params(1, 32768, 48, 128, num_seqs=16)):
         assert ssd.workspace_size(p) > 0
