@@ -159,6 +159,150 @@ def _ptr(t) -> Optional[int]:
     return None if t is None else int(t.data_ptr())
 
 
+# ---------------------------------------------------------------- argument checks
+# The kernels dereference every pointer they are given, over the extent the
+# shapes imply: a host tensor, a tensor on another GPU, a short buffer or a
+# strided view would be read or written out of bounds on the device.  These
+# checks look at tensor metadata only (dtype, shape, contiguity, device), so
+# they run before anything is launched.
+
+def _check(name, t, dev, dtype, shape=None, required=False):
+    """`t` (None when optional) must be a contiguous `dtype` tensor on `dev`
+    with exactly `shape` (when given)."""
+    if t is None:
+        if required:
+            raise ValueError(f"{name} is required")
+        return
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.device != dev:
+        raise ValueError(f"{name} must be on {dev}, got {t.device}")
+
+
+def _io_dtype(x):
+    import torch
+    if x.dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError(f"x must be bfloat16 or float32, got {x.dtype}")
+    return x.dtype
+
+
+def _check_workspace(workspace, dev):
+    if workspace is not None and (not workspace.is_contiguous() or workspace.device != dev):
+        raise ValueError(f"workspace must be a contiguous tensor on {dev}")
+
+
+def _check_sequence_inputs(x, dt, A_log, B, cu_seqlens):
+    """Shared checks of x, dt, A_log, B and cu_seqlens; returns
+    (b, T, H, P, G, N, nseq)."""
+    import torch
+    io = _io_dtype(x)
+    if x.dim() != 4:
+        raise ValueError(f"x must be (batch, seqlen, nheads, headdim), got {tuple(x.shape)}")
+    if B is None or B.dim() != 4:
+        raise ValueError("B must be (batch, seqlen, ngroups, dstate)")
+    dev = x.device
+    b, T, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    _check("x", x, dev, io)
+    _check("dt", dt, dev, io, (b, T, H), required=True)
+    _check("B", B, dev, io, (b, T, G, N))
+    _check("A_log", A_log, dev, torch.float32, (H,), required=True)
+    nseq = b
+    if cu_seqlens is not None:
+        _check("cu_seqlens", cu_seqlens, dev, torch.int32)
+        if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
+            raise ValueError("cu_seqlens must be 1-D with nseq + 1 >= 2 entries")
+        nseq = cu_seqlens.numel() - 1
+    return b, T, H, P, G, N, nseq
+
+
+def _validate_fwd(x, dt, A_log, B, C, D=None, initial_states=None, cu_seqlens=None, y=None, final_states=None,
+                  workspace=None, z=None, norm_weight=None, norm_bias=None):
+    """Every tensor argument of ssd_fwd (metadata only); returns nseq."""
+    import torch
+    b, T, H, P, G, N, nseq = _check_sequence_inputs(x, dt, A_log, B, cu_seqlens)
+    dev, io = x.device, x.dtype
+    _check("C", C, dev, io, (b, T, G, N), required=True)
+    _check("D", D, dev, torch.float32, (H,))
+    _check("initial_states", initial_states, dev, torch.float32, (nseq, H, P, N))
+    _check("y", y, dev, io, (b, T, H, P))
+    _check("final_states", final_states, dev, torch.float32, (nseq, H, P, N))
+    _check_workspace(workspace, dev)
+    if z is None:
+        if norm_weight is not None or norm_bias is not None:
+            raise ValueError("norm_weight and norm_bias are used only together with z")
+        return nseq
+    _check("z", z, dev, io, (b, T, H, P))
+    _check("norm_weight", norm_weight, dev, torch.float32, required=True)
+    _check("norm_bias", norm_bias, dev, torch.float32)
+    for name, t in (("norm_weight", norm_weight), ("norm_bias", norm_bias)):
+        if t is not None and t.numel() != H * P:
+            raise ValueError(f"{name} must hold nheads * headdim = {H * P} values, got {t.numel()}")
+    return nseq
+
+
+def _validate_summary(x, dt, A_log, B, cu_seqlens=None, workspace=None):
+    """Every tensor argument of ssd_fwd_summary; returns nseq."""
+    nseq = _check_sequence_inputs(x, dt, A_log, B, cu_seqlens)[-1]
+    _check_workspace(workspace, x.device)
+    return nseq
+
+
+def _validate_bwd(x, dt, A_log, B, C, D, dy, initial_states=None, cu_seqlens=None, dfinal_states=None,
+                  workspace=None):
+    """Every tensor argument of ssd_bwd; returns nseq."""
+    import torch
+    b, T, H, P, G, N, nseq = _check_sequence_inputs(x, dt, A_log, B, cu_seqlens)
+    dev, io = x.device, x.dtype
+    _check("C", C, dev, io, (b, T, G, N), required=True)
+    _check("D", D, dev, torch.float32, (H,))
+    _check("dy", dy, dev, io, (b, T, H, P), required=True)
+    _check("initial_states", initial_states, dev, torch.float32, (nseq, H, P, N))
+    _check("dfinal_states", dfinal_states, dev, torch.float32, (nseq, H, P, N))
+    _check_workspace(workspace, dev)
+    return nseq
+
+
+def _validate_decode(x, dt, A_log, B, C, D, state, y=None):
+    """Every tensor argument of ssd_decode_step."""
+    import torch
+    io = _io_dtype(x)
+    if x.dim() != 3:
+        raise ValueError(f"x must be (batch, nheads, headdim), got {tuple(x.shape)}")
+    if B is None or B.dim() != 3:
+        raise ValueError("B must be (batch, ngroups, dstate)")
+    dev = x.device
+    b, H, P = x.shape
+    G, N = B.shape[1], B.shape[2]
+    _check("x", x, dev, io)
+    _check("dt", dt, dev, io, (b, H), required=True)
+    _check("B", B, dev, io, (b, G, N))
+    _check("C", C, dev, io, (b, G, N), required=True)
+    _check("A_log", A_log, dev, torch.float32, (H,), required=True)
+    _check("D", D, dev, torch.float32, (H,))
+    _check("state", state, dev, torch.float32, (b, H, P, N), required=True)
+    _check("y", y, dev, io, (b, H, P))
+
+
+def _validate_combine(end_states_all, logdecay_all, rank, initial_states=None, out=None):
+    """Every tensor argument of ssd_state_combine."""
+    import torch
+    if end_states_all is None or end_states_all.dim() != 5:
+        raise ValueError("end_states_all must be (world, nseq, nheads, headdim, dstate)")
+    dev = end_states_all.device
+    world, nseq, H, P, N = end_states_all.shape
+    _check("end_states_all", end_states_all, dev, torch.float32)
+    _check("logdecay_all", logdecay_all, dev, torch.float32, (world, nseq, H), required=True)
+    _check("initial_states", initial_states, dev, torch.float32, (nseq, H, P, N))
+    _check("out", out, dev, torch.float32, (nseq, H, P, N))
+    if not 0 <= int(rank) <= world:
+        raise ValueError(f"rank must be in 0..{world}, got {rank}")
+
+
 def _stream_handle(stream) -> Optional[int]:
     import torch
     if stream is None:
@@ -204,29 +348,16 @@ def ssd_fwd(x, dt, A_log, B, C, D=None, chunk_len: int = 256, initial_states=Non
     dev = x.device
     if dev.type != "cuda":
         raise ValueError("ssd_fwd runs on CUDA tensors only")
-    for name, t in (("x", x), ("dt", dt), ("B", B), ("C", C)):
-        if t.dtype != x.dtype or not t.is_contiguous() or t.device != dev:
-            raise ValueError(f"{name} must be a contiguous {x.dtype} tensor on {dev}")
-    for name, t in (("A_log", A_log), ("D", D), ("initial_states", initial_states)):
-        if t is not None and (t.dtype != torch.float32 or not t.is_contiguous() or t.device != dev):
-            raise ValueError(f"{name} must be a contiguous float32 tensor on {dev}")
-    if cu_seqlens is not None and (cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_contiguous()):
-        raise ValueError("cu_seqlens must be a contiguous int32 tensor")
-    if x.dim() != 4 or dt.shape != x.shape[:3] or B.shape != C.shape or B.shape[:2] != x.shape[:2]:
-        raise ValueError("shape mismatch between x, dt, B, C")
+    nseq = _validate_fwd(x, dt, A_log, B, C, D, initial_states, cu_seqlens, y, final_states, workspace, z,
+                         norm_weight, norm_bias)
     p = params_for(x, B, chunk_len, cu_seqlens, dt_softplus, path)
     b, T, H, P = x.shape
     N = B.shape[3]
-    nseq = p.num_seqs if p.num_seqs > 0 else b
     if y is None:
         y = torch.empty_like(x)
     want_final = return_final_states or final_states is not None
     if want_final and final_states is None:
         final_states = torch.empty((nseq, H, P, N), dtype=torch.float32, device=dev)
-    if initial_states is not None and tuple(initial_states.shape) != (nseq, H, P, N):
-        raise ValueError(f"initial_states must have shape {(nseq, H, P, N)}")
-    if final_states is not None and tuple(final_states.shape) != (nseq, H, P, N):
-        raise ValueError(f"final_states must have shape {(nseq, H, P, N)}")
     need = int(lib.ssd_fwd_workspace_size(ctypes.byref(p)))
     if need == 0:
         raise SsdError(-2 if lib.ssd_fwd_resolved_path(ctypes.byref(p)) == -1 else -1, "ssd_fwd_workspace_size")
@@ -237,14 +368,6 @@ def ssd_fwd(x, dt, A_log, B, C, D=None, chunk_len: int = 256, initial_states=Non
             _ptr(initial_states), _ptr(cu_seqlens), _ptr(y), _ptr(final_states),
             _ptr(workspace), workspace.numel() * workspace.element_size(), st)
     if z is not None:
-        for name, t in (("z", z),):
-            if t.dtype != x.dtype or not t.is_contiguous() or t.shape != x.shape or t.device != dev:
-                raise ValueError(f"{name} must be a contiguous {x.dtype} tensor shaped like x")
-        for name, t in (("norm_weight", norm_weight), ("norm_bias", norm_bias)):
-            if t is not None and (t.dtype != torch.float32 or not t.is_contiguous() or t.numel() != H * P):
-                raise ValueError(f"{name} must be a contiguous float32 tensor of nheads * headdim values")
-        if norm_weight is None:
-            raise ValueError("norm_weight is required with z")
         rc = lib.ssd_fwd_gated_norm(ctypes.byref(p), _ptr(x), _ptr(dt), _ptr(A_log), _ptr(B), _ptr(C), _ptr(D),
                                     _ptr(initial_states), _ptr(cu_seqlens), _ptr(z), _ptr(norm_weight),
                                     _ptr(norm_bias), float(norm_eps), _ptr(y), _ptr(final_states),
@@ -272,13 +395,10 @@ def ssd_fwd_summary(x, dt, A_log, B, chunk_len: int = 256, cu_seqlens=None, dt_s
     dev = x.device
     if dev.type != "cuda":
         raise ValueError("ssd_fwd_summary runs on CUDA tensors only")
-    for name, t in (("x", x), ("dt", dt), ("B", B)):
-        if t.dtype != x.dtype or not t.is_contiguous() or t.device != dev:
-            raise ValueError(f"{name} must be a contiguous {x.dtype} tensor on {dev}")
+    nseq = _validate_summary(x, dt, A_log, B, cu_seqlens, workspace)
     p = params_for(x, B, chunk_len, cu_seqlens, dt_softplus, path)
     b, T, H, P = x.shape
     N = B.shape[3]
-    nseq = p.num_seqs if p.num_seqs > 0 else b
     S = torch.empty((nseq, H, P, N), dtype=torch.float32, device=dev)
     L = torch.empty((nseq, H), dtype=torch.float32, device=dev)
     need = int(lib.ssd_fwd_summary_workspace_size(ctypes.byref(p)))
@@ -304,13 +424,10 @@ def ssd_state_combine(end_states_all, logdecay_all, rank: int, initial_states=No
     the state entering worker `rank` (rank == world: after the last piece)."""
     import torch
     lib = library()
+    if end_states_all.device.type != "cuda":
+        raise ValueError("ssd_state_combine runs on CUDA tensors only")
+    _validate_combine(end_states_all, logdecay_all, rank, initial_states, out)
     world, nseq, H, P, N = end_states_all.shape
-    for name, t in (("end_states_all", end_states_all), ("logdecay_all", logdecay_all),
-                    ("initial_states", initial_states)):
-        if t is not None and (t.dtype != torch.float32 or not t.is_contiguous() or t.device.type != "cuda"):
-            raise ValueError(f"{name} must be a contiguous float32 CUDA tensor")
-    if tuple(logdecay_all.shape) != (world, nseq, H):
-        raise ValueError("logdecay_all must be (world, nseq, nheads)")
     if out is None:
         out = torch.empty((nseq, H, P, N), dtype=torch.float32, device=end_states_all.device)
     rc = lib.ssd_state_combine(int(world), int(rank), int(nseq), int(H), int(P), int(N), _ptr(end_states_all),
@@ -331,19 +448,10 @@ def ssd_bwd(x, dt, A_log, B, C, D, dy, initial_states=None, cu_seqlens=None, dfi
     dev = x.device
     if dev.type != "cuda":
         raise ValueError("ssd_bwd runs on CUDA tensors only")
-    for name, t in (("x", x), ("dt", dt), ("B", B), ("C", C), ("dy", dy)):
-        if t.dtype != x.dtype or not t.is_contiguous() or t.device != dev:
-            raise ValueError(f"{name} must be a contiguous {x.dtype} tensor on {dev}")
-    for name, t in (("A_log", A_log), ("D", D), ("initial_states", initial_states),
-                    ("dfinal_states", dfinal_states)):
-        if t is not None and (t.dtype != torch.float32 or not t.is_contiguous() or t.device != dev):
-            raise ValueError(f"{name} must be a contiguous float32 tensor on {dev}")
-    if dy.shape != x.shape:
-        raise ValueError("dy must have x's shape")
+    nseq = _validate_bwd(x, dt, A_log, B, C, D, dy, initial_states, cu_seqlens, dfinal_states, workspace)
     p = params_for(x, B, 256, cu_seqlens, dt_softplus, "auto")
     b, T, H, P = x.shape
     G, N = B.shape[2], B.shape[3]
-    nseq = p.num_seqs if p.num_seqs > 0 else b
     f32 = dict(dtype=torch.float32, device=dev)
     out = {"dx": torch.empty(x.shape, **f32), "ddt": torch.empty(dt.shape, **f32),
            "dA_log": torch.empty(H, **f32), "dB": torch.empty(B.shape, **f32), "dC": torch.empty(C.shape, **f32),
@@ -382,18 +490,9 @@ def ssd_decode_step(x, dt, A_log, B, C, D, state, y=None, dt_softplus: bool = Tr
     dev = x.device
     if dev.type != "cuda":
         raise ValueError("ssd_decode_step runs on CUDA tensors only")
-    if x.dtype not in (torch.bfloat16, torch.float32):
-        raise TypeError(f"x must be bfloat16 or float32, got {x.dtype}")
-    for name, t in (("x", x), ("dt", dt), ("B", B), ("C", C)):
-        if t.dtype != x.dtype or not t.is_contiguous() or t.device != dev:
-            raise ValueError(f"{name} must be a contiguous {x.dtype} tensor on {dev}")
-    for name, t in (("A_log", A_log), ("D", D), ("state", state)):
-        if t is not None and (t.dtype != torch.float32 or not t.is_contiguous() or t.device != dev):
-            raise ValueError(f"{name} must be a contiguous float32 tensor on {dev}")
+    _validate_decode(x, dt, A_log, B, C, D, state, y)
     b, H, P = x.shape
     G, N = B.shape[1], B.shape[2]
-    if tuple(dt.shape) != (b, H) or tuple(C.shape) != (b, G, N) or tuple(state.shape) != (b, H, P, N):
-        raise ValueError("shape mismatch between x, dt, B, C, state")
     if y is None:
         y = torch.empty_like(x)
     p = SsdStepParams(int(b), int(H), int(P), int(N), int(G), DTYPES["bf16" if x.dtype == torch.bfloat16 else "f32"],
