@@ -37,3 +37,57 @@ def test_traffic_figures_follow_code_not_comments():
     assert bench._code_only(a) != bench._code_only(c)
     h = bench.kernel_source_hash()
     assert len(h) == 16 and h == bench.kernel_source_hash()
+
+
+def test_timed_loop_with_and_without_flush(monkeypatch):
+    """Forward.timed runs warm-up + timed steps with the L2 flush before each,
+    or with none (the warm-L2 figures), and a device error during the warm-L2
+    run ends up in the JSON line instead of ending the bench.  Fake CUDA
+    events stand in for the GPU."""
+    import types
+    import torch
+    sys.path.insert(0, ROOT)
+    import bench
+
+    class Ev:
+        clock = 0
+
+        def __init__(self, enable_timing=False):
+            self.t = None
+
+        def record(self, stream=None):
+            Ev.clock += 1
+            self.t = Ev.clock
+
+        def elapsed_time(self, other):
+            return float(other.t - self.t)
+
+    class Flush:
+        def __init__(self):
+            self.n = 0
+
+        def zero_(self):
+            self.n += 1
+
+    monkeypatch.setattr(torch.cuda, "Event", Ev)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
+    fw = object.__new__(bench.Forward)
+    calls = []
+    fw.stream = None
+    fw.step = lambda events=None: calls.append(events)
+    fw.status = lambda: 0
+    fw.ssd = types.SimpleNamespace(SsdError=lambda rc, what: RuntimeError(f"{what}: {rc}"))
+    fl = Flush()
+    s, c, m, _ = fw.timed(4, 3, fl)
+    assert fl.n == 7 and len(calls) == 7 and len(s) == len(c) == len(m) == 4
+    assert all(e is not None and len(e) == 3 for e in calls[3:]) and all(e is None for e in calls[:3])
+    assert all(v > 0 for v in s + c + m)
+    calls.clear()
+    s, c, m, _ = fw.timed(5, 3, None)
+    assert len(calls) == 8 and len(s) == 5 and fl.n == 7
+    w = bench.warm_l2_stats(fw, 6)
+    assert w["steps"] == 6 and set(w) == {"steps", "step_ms", "compute_ms", "output_pass_ms"}
+    assert w["step_ms"]["min"] > 0
+    fw.status = lambda: -4
+    w = bench.warm_l2_stats(fw, 6)
+    assert set(w) == {"error"} and "-4" in w["error"]
