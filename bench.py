@@ -71,6 +71,16 @@ def algorithmic_flops(inp: dict, block_len: int) -> int:
     return int(tokens * (H * (4 * P * N + Q * P) + G * Q * N))
 
 
+def full_tile_flops(inp: dict, block_len: int) -> int:
+    """The same with whole Q x Q diagonal tiles (no causal halving), the work a
+    tiled evaluation issues: per token H * (4PN + 2QP) + 2GQN."""
+    x, B = inp["x"], inp["B"]
+    tokens = x.shape[0] * x.shape[1]
+    H, P, G, N = x.shape[2], x.shape[3], B.shape[2], B.shape[3]
+    Q = block_len
+    return int(tokens * (H * (4 * P * N + 2 * Q * P) + 2 * G * Q * N))
+
+
 def _code_only(text: str) -> str:
     """CUDA/C++ source without comments and with whitespace collapsed, so that
     editing a comment does not change the hash (the sources contain no comment
@@ -531,6 +541,7 @@ def run_ours(args):
             "step_ms": _stats(step_ms), "compute_ms": _stats(comp_ms), "output_pass_ms": _stats(main_ms),
             "roofline": roof,
             "tflops": flops / (ms * 1e-3) / 1e12, "flops_block_len": block_len,
+            "tflops_full_tile": full_tile_flops(inp, block_len) / (ms * 1e-3) / 1e12,
             "check": check,
             "cpu_baseline": cpu,
             "e2e": {"value": whole_job_throughput(tokens, world, e2e), "unit": "tokens/s", "h2d_bytes_per_step": h2d,

@@ -91,3 +91,20 @@ def test_timed_loop_with_and_without_flush(monkeypatch):
     fw.status = lambda: -4
     w = bench.warm_l2_stats(fw, 6)
     assert set(w) == {"error"} and "-4" in w["error"]
+
+
+def test_accounting_of_the_benchmark_workloads():
+    """Bytes and FLOPs per forward, worked out by hand from the shapes:
+    2.7B-shaped layer (8 x 2048 tokens, H 80, P 64, N 128, G 1, bf16):
+    x + y = 2 * 167,772,160 B, dt 2,621,440 B, B + C = 2 * 4,194,304 B;
+    16K GVA (H 32, P 64, N 256, G 8) adds 32 * 64 * 256 = 524,288 floats of final state."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import ssd_inputs
+    inp = ssd_inputs.make_inputs(ssd_inputs.workload("mamba2_2p7b"), seed=0)
+    assert bench.algorithmic_bytes(inp) == 2 * 167_772_160 + 2_621_440 + 2 * 4_194_304
+    tok = 8 * 2048
+    assert bench.algorithmic_flops(inp, 128) == tok * (80 * (4 * 64 * 128 + 128 * 64) + 128 * 128)
+    assert bench.full_tile_flops(inp, 256) == tok * (80 * (4 * 64 * 128 + 2 * 256 * 64) + 2 * 256 * 128)
+    inp = ssd_inputs.make_inputs(ssd_inputs.workload("long16k_gva"), seed=0)
+    assert bench.algorithmic_bytes(inp) == 2 * 67_108_864 + 1_048_576 + 2 * 67_108_864 + 4 * 524_288
