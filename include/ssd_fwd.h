@@ -105,8 +105,12 @@ typedef struct ssd_fwd_params {
 } ssd_fwd_params;
 
 /* Bytes of device workspace ssd_fwd needs for these parameters (0 on invalid
- * parameters).  The workspace must be 256-byte aligned; its contents need no
- * initialisation and may be reused by the next call on the same stream. */
+ * parameters), for the device current at the time of the query: the schedule
+ * of equal-length rows depends on that device's SM count (at most 148 are
+ * used), so ask with the device current that the call will run on.  ssd_fwd
+ * recomputes the size and returns SSD_ERR_INVALID_ARG for a smaller workspace.
+ * The workspace must be 256-byte aligned; its contents need no initialisation
+ * and may be reused by the next call on the same stream. */
 SSD_API size_t ssd_fwd_workspace_size(const ssd_fwd_params *p);
 
 /* SSD forward.  D, initial_states, cu_seqlens and final_states may be NULL

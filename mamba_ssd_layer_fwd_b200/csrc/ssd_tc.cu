@@ -1597,8 +1597,12 @@ struct TcPlanShape {
     bool segmented;
 };
 
-// The work split is a pure function of the parameters (the workspace size must
-// not depend on which GPU answers), sized for the B200's 148 SMs.
+// The split of packed sequences is a pure function of the parameters, sized
+// for the B200's 148 SMs.  The schedule of equal-length rows (uniform_plan)
+// also takes min(148, SMs of the current device): its segmented launch needs
+// every CTA resident at once.  So the workspace size is that of the device
+// current when it is asked for; ssd_fwd recomputes it and rejects a smaller
+// workspace.
 constexpr int kPlanSMs = 148;
 
 // Segment count (1 = no cut) with the smallest modelled makespan for `rows`
